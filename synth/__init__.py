@@ -1,0 +1,239 @@
+"""Seeded synthetic inputs for the GRINQH decode path (shared by tests and bench).
+
+This module holds no step of the method itself: it draws weights and
+activations, applies the *base* quantizer that GRINQH is layered on
+(round-to-nearest, 8-bit asymmetric, 128-row groups, fp16 scale/zero -- the
+"GRINQH-8b-RTN" rows of the GRINQH notes' main results table), and picks
+static thresholds from activation quantiles the way the offline calibration
+of "Key design 1" describes.  The precision assignment, row lists, bit-plane
+packing, reconstruction and GEMV live in the CUDA library and, independently,
+in the oracle.
+
+All randomness comes from ``numpy.random.default_rng``; a case is identified
+by (config id, layer, call).  Config 0 uses seed 0 directly.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+
+import numpy as np
+
+GROUP = 128
+
+# Level fractions (b = 0, 2, 4, 6, 8) for a target mean bit width at b_max = 8.
+# The pages give no table; these follow the sparsity ablation of the GRINQH
+# notes ("Key findings": >= 20% zero-bit channels help at 2-3 bits, smoother
+# allocation is better near 4 bits) and hit the target mean exactly.
+LEVEL_FRACTIONS_BMAX8 = {
+    2.0: (0.40, 0.35, 0.15, 0.05, 0.05),
+    3.0: (0.20, 0.40, 0.20, 0.10, 0.10),
+    3.3: (0.20, 0.30, 0.25, 0.15, 0.10),
+    4.0: (0.10, 0.25, 0.35, 0.15, 0.15),
+}
+# b_max = 4 mixed mode (b = 0, 2, 4): 2.4 bits.
+LEVEL_FRACTIONS_BMAX4_MIX = (0.20, 0.40, 0.40)
+
+
+def rng(config_id: int, layer: int = 0, call: int = 0) -> np.random.Generator:
+    if config_id == 0 and layer == 0 and call == 0:
+        return np.random.default_rng(0)
+    return np.random.default_rng(np.random.SeedSequence([config_id, layer, call]))
+
+
+def gaussian_weights(g: np.random.Generator, d_in: int, d_out: int,
+                     std: float = 0.02) -> np.ndarray:
+    """W ~ N(0, std^2), fp32, shape [d_in, d_out] (reduction dimension first)."""
+    return (g.standard_normal((d_in, d_out), dtype=np.float32) * np.float32(std))
+
+
+def rtn_quantize(W: np.ndarray, bits: int = 8, group: int = GROUP):
+    """Base RTN quantizer: per (group of `group` rows, output channel)
+    s = (max - min) / (2^bits - 1), z = min, both rounded to fp16, and
+    q = clamp(round_half_even((w - z16) / s16), 0, 2^bits - 1) in fp64
+    (q = 0 where s16 == 0).  Returns q uint8 [d_in, d_out], s, z fp16 [G, d_out].
+    """
+    d_in, d_out = W.shape
+    assert d_in % group == 0
+    G = d_in // group
+    qmax = (1 << bits) - 1
+    q = np.empty((d_in, d_out), np.uint8)
+    s16 = np.empty((G, d_out), np.float16)
+    z16 = np.empty((G, d_out), np.float16)
+    for g in range(G):
+        blk = W[g * group:(g + 1) * group].astype(np.float64)
+        lo = blk.min(axis=0)
+        hi = blk.max(axis=0)
+        s16[g] = ((hi - lo) / qmax).astype(np.float16)
+        z16[g] = lo.astype(np.float16)
+        sv = s16[g].astype(np.float64)
+        zv = z16[g].astype(np.float64)
+        with np.errstate(divide="ignore", invalid="ignore"):
+            code = np.rint((blk - zv) / sv)
+        code = np.where(sv == 0.0, 0.0, code)
+        q[g * group:(g + 1) * group] = np.clip(code, 0, qmax).astype(np.uint8)
+    return q, s16, z16
+
+
+def activations(g: np.random.Generator, d_in: int, dist: str = "normal",
+                outlier_frac: float = 0.01, outlier_scale: float = 20.0) -> np.ndarray:
+    """Decode-time input vector, fp16.
+
+    ``normal``: N(0, 1) with exactly round(outlier_frac * d_in) distinct
+    entries, chosen uniformly, multiplied by ``outlier_scale`` before the fp16
+    cast.  ``student_t``: Student-t with 3 degrees of freedom (heavy tails),
+    no planted outliers.
+    """
+    if dist == "normal":
+        x = g.standard_normal(d_in)
+        n_out = int(round(outlier_frac * d_in))
+        if n_out:
+            idx = g.choice(d_in, size=n_out, replace=False)
+            x[idx] *= outlier_scale
+    elif dist == "student_t":
+        x = g.standard_t(3.0, size=d_in)
+    else:
+        raise ValueError(dist)
+    return x.astype(np.float16)
+
+
+def quantile_thresholds(abs_pool: np.ndarray, fractions) -> np.ndarray:
+    """Static Theta from |x| quantiles: theta_k = sorted(|x|)[floor(c_k * n)],
+    c_k = fraction of channels below level k.  Returns fp32 [P]."""
+    a = np.sort(np.abs(np.asarray(abs_pool, np.float32)).ravel())
+    n = a.shape[0]
+    c = np.cumsum(np.asarray(fractions, np.float64))[:-1]
+    theta = np.empty(len(c), np.float32)
+    for k, ck in enumerate(c):
+        idx = int(np.floor(ck * n + 1e-9))
+        theta[k] = a[idx] if idx < n else np.float32(np.inf)
+    return theta
+
+
+def uniform_thresholds(b: int, b_max: int) -> np.ndarray:
+    """Theta that puts every channel at bit width b: theta_1..theta_{b/2} = 0,
+    the rest +inf."""
+    P = b_max // 2
+    theta = np.full(P, np.inf, np.float32)
+    theta[: b // 2] = 0.0
+    return theta
+
+
+def level_fractions(target_bits: float, b_max: int = 8):
+    if b_max == 8:
+        return LEVEL_FRACTIONS_BMAX8[target_bits]
+    if b_max == 4 and abs(target_bits - 2.4) < 1e-9:
+        return LEVEL_FRACTIONS_BMAX4_MIX
+    raise KeyError((target_bits, b_max))
+
+
+@dataclass
+class Linear:
+    """One decode GEMV: its shape, base width and input recipe."""
+    name: str
+    d_in: int
+    d_out: int
+    b_max: int = 8
+    target_bits: float | None = 3.0   # None: uniform width `uniform_b`
+    uniform_b: int | None = None
+    dist: str = "normal"
+    config_id: int = 1
+    layer: int = 0
+    calib_draws: int = 0              # >0: Theta from that many pooled draws
+    extra: dict = field(default_factory=dict)
+
+
+@dataclass
+class Case:
+    """Generated host-side inputs of one Linear."""
+    lin: Linear
+    q: np.ndarray
+    s: np.ndarray
+    z: np.ndarray
+    x: np.ndarray
+    theta: np.ndarray
+
+
+def make_theta(lin: Linear, x: np.ndarray) -> np.ndarray:
+    if lin.target_bits is None:
+        return uniform_thresholds(lin.uniform_b, lin.b_max)
+    fr = level_fractions(lin.target_bits, lin.b_max)
+    if lin.calib_draws:
+        pool = np.stack([activations(rng(lin.config_id, lin.layer, 10_000 + c), lin.d_in, lin.dist)
+                         for c in range(lin.calib_draws)])
+        return quantile_thresholds(np.abs(pool.astype(np.float32)), fr)
+    return quantile_thresholds(np.abs(x.astype(np.float32)), fr)
+
+
+def make_case(lin: Linear, call: int = 0, weights_rng_call: int = 0) -> Case:
+    g = rng(lin.config_id, lin.layer, weights_rng_call)
+    W = gaussian_weights(g, lin.d_in, lin.d_out)
+    q, s, z = rtn_quantize(W, lin.b_max)
+    del W
+    gx = g if call == weights_rng_call else rng(lin.config_id, lin.layer, call)
+    x = activations(gx, lin.d_in, lin.dist)
+    theta = make_theta(lin, x)
+    return Case(lin, q, s, z, x, theta)
+
+
+def make_x(lin: Linear, call: int) -> np.ndarray:
+    """A fresh activation vector for call `call` of a Linear (weights unchanged)."""
+    return activations(rng(lin.config_id, lin.layer, 1_000_000 + call), lin.d_in, lin.dist)
+
+
+# ---- The five workloads -------------------------------------------------------
+
+def config0():
+    """Parity case: 512 -> 512, levels 20/30/25/15/10 % (3.3 bits), seed 0."""
+    return [Linear("single_512", 512, 512, target_bits=3.3, config_id=0)]
+
+
+QWEN3_8B = [("q_proj", 4096, 4096), ("gate_proj", 4096, 12288),
+            ("up_proj", 4096, 12288), ("down_proj", 12288, 4096)]
+
+
+def config1(bits=(2.0, 3.0, 4.0)):
+    """Qwen3-8B-shaped projections at batch 1, Theta from |x| quantiles."""
+    out = []
+    for bi, tb in enumerate(bits):
+        for li, (n, di, do) in enumerate(QWEN3_8B):
+            out.append(Linear(f"{n}@{tb:g}b", di, do, target_bits=tb, config_id=1,
+                              layer=10 * bi + li))
+    return out
+
+
+def config2():
+    """Uniform-width sweep on 4096 -> 14336 (Llama-3-8B up_proj shape)."""
+    out = [Linear(f"up14336_u{b}", 4096, 14336, target_bits=None, uniform_b=b, config_id=2,
+                  layer=0) for b in (2, 4, 6, 8)]
+    out += [Linear(f"up14336_bmax4_u{b}", 4096, 14336, b_max=4, target_bits=None, uniform_b=b,
+                   config_id=2, layer=1) for b in (2, 4)]
+    out.append(Linear("up14336_bmax4_mix", 4096, 14336, b_max=4, target_bits=2.4, config_id=2,
+                      layer=1))
+    return out
+
+
+def config3(bits=(2.0, 3.0, 4.0)):
+    """70B-class shapes, Student-t inputs, Theta from 128 pooled calibration draws."""
+    out = []
+    for bi, tb in enumerate(bits):
+        for li, (n, di, do) in enumerate([("up70b", 8192, 28672), ("down70b", 28672, 8192)]):
+            out.append(Linear(f"{n}@{tb:g}b", di, do, target_bits=tb, dist="student_t",
+                              config_id=3, layer=10 * bi + li, calib_draws=128))
+    return out
+
+
+LLAMA3_8B = [("q", 4096, 4096), ("k", 4096, 1024), ("v", 4096, 1024), ("o", 4096, 4096),
+             ("gate", 4096, 14336), ("up", 4096, 14336), ("down", 14336, 4096)]
+
+
+def config4(n_layers: int = 32):
+    """Full decode step: 32 Llama-3-8B layers x 7 linears, 3 bits each."""
+    out = []
+    for layer in range(n_layers):
+        for li, (n, di, do) in enumerate(LLAMA3_8B):
+            out.append(Linear(f"L{layer}.{n}", di, do, target_bits=3.0, config_id=4,
+                              layer=100 * layer + li))
+    return out
+
+
+CONFIGS = {0: config0, 1: config1, 2: config2, 3: config3, 4: config4}
