@@ -1,0 +1,553 @@
+#!/usr/bin/env python
+"""Throughput of the GRINQH batch-1 decode GEMV on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload qwen3-8b-proj|uniform-sweep|70b|llama3-8b-step]
+
+A step is one pass of the whole decode path -- grinqh_assign then
+grinqh_gemv -- over one token's inputs for every linear of the workload.  The
+default workload is the Qwen3-8B-shaped projection set at batch 1 (q_proj
+4096->4096, gate/up 4096->12288, down 12288->4096) at 2.0, 3.0 and 4.0
+effective bits: 12 GEMVs per step, each with its own packed weights (504 MB of
+planes, ~200 MB read per step, so consecutive steps do not hit in the 126 MB
+L2).  Inputs are seeded synthetic: W ~ N(0, 0.02) quantized by 8-bit RTN,
+x ~ N(0, 1) with 1% outliers x20, a fresh x per step from a pool of 8, and
+static thresholds calibrated on 128 pooled draws.
+
+The headline value is effective HBM bandwidth: the minimum bytes the method
+must move (planes of the assigned widths, s/z of active groups, x, y) per
+step, divided by the device time of the step.  One JSON line is printed by
+rank 0.  With --gpus N > 1 (under torchrun) every rank runs its own replica of
+the workload (weak scaling, no collective on the data path); the step time is
+the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "µs per decode GEMV and effective HBM GB/s (fraction of B200 peak) vs eff. bits"
+UNIT = "GB/s"
+L2_BYTES = 126 * 1024 * 1024
+N_POOL = 8
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--warmup", type=int, default=100)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="qwen3-8b-proj",
+                    choices=["qwen3-8b-proj", "uniform-sweep", "70b", "llama3-8b-step"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-cases", action="store_true", help="skip the per-GEMV cold-L2 table")
+    return ap.parse_args(argv)
+
+
+def workload_specs(name):
+    if name == "qwen3-8b-proj":
+        return synth.config1()
+    if name == "uniform-sweep":
+        return synth.config2()
+    if name == "70b":
+        return synth.config3()
+    if name == "llama3-8b-step":
+        return synth.config4()
+    raise ValueError(name)
+
+
+def min_bytes(b: np.ndarray, d_out: int, include_x: bool = True) -> int:
+    """Algorithmic bytes of one decode GEMV: the planes of the assigned widths,
+    fp16 s and z of every group with an active row, x (fp16) and y (fp32)."""
+    d_in = b.shape[0]
+    planes = int(b.astype(np.int64).sum()) * d_out // 8
+    g_act = int((b.reshape(-1, 128) > 0).any(axis=1).sum())
+    return planes + 4 * d_out * g_act + (2 * d_in if include_x else 0) + 4 * d_out
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            mp = json.load(f)
+        return float(mp["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ---- clocks during the timed region ---------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str | None):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.t0 = None
+
+    def start(self):
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+               "-lms", "20"]
+        if self.gpu_id:
+            cmd += ["-i", self.gpu_id]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                         text=True)
+        except Exception:
+            self.proc = None
+        self.t0 = time.time()
+
+    def stop(self):
+        if self.proc is None:
+            return []
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except Exception:
+            self.proc.kill()
+            out = ""
+        rows = []
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        return rows
+
+    @staticmethod
+    def summarize(rows):
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+
+        def num(v):
+            try:
+                return float(v)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        smax = [num(r[2]) for r in rows if num(r[2]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.strip() == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": reasons, "samples": len(rows),
+                "power_w_max": max((num(r[3]) or 0.0) for r in rows)}
+
+
+# ---- the CUDA path ------------------------------------------------------------------
+
+class Workload:
+    """Device-resident layers, input pools and captured step graphs."""
+
+    def __init__(self, specs, device, rank):
+        import torch
+        from input_adaptive_bit_b200.layer import GrinqhLinear
+        self.torch = torch
+        self.device = device
+        self.specs = specs
+        self.layers, self.thetas = [], []
+        cache = {}
+        for spec in specs:
+            # base codes are drawn once per distinct projection (name without the
+            # bit-target / layer prefix); every linear still gets its own packed copy
+            proj = (spec.d_in, spec.d_out, spec.b_max, spec.name.split("@")[0].split(".")[-1])
+            if proj not in cache:
+                g = synth.rng(spec.config_id, 1000 + len(cache), rank)
+                W = synth.gaussian_weights(g, spec.d_in, spec.d_out)
+                cache[proj] = synth.rtn_quantize(W, spec.b_max)
+                del W
+            q, s, z = cache[proj]
+            self.layers.append(GrinqhLinear(q, s, z, spec.b_max, device=device))
+            calib = synth.Linear(spec.name, spec.d_in, spec.d_out, spec.b_max, spec.target_bits,
+                                 spec.uniform_b, spec.dist, spec.config_id, spec.layer,
+                                 calib_draws=128 if spec.target_bits is not None else 0)
+            x0 = synth.activations(synth.rng(spec.config_id, spec.layer, 0), spec.d_in, spec.dist)
+            self.thetas.append(torch.from_numpy(synth.make_theta(calib, x0)).to(device))
+        del cache
+        # x pool: [N_POOL][sum d_in] fp16, host (pinned) and device copies
+        self.offsets = np.cumsum([0] + [s.d_in for s in specs])
+        self.y_offsets = np.cumsum([0] + [s.d_out for s in specs])
+        xs = np.zeros((N_POOL, self.offsets[-1]), np.float16)
+        for k in range(N_POOL):
+            for j, spec in enumerate(specs):
+                xs[k, self.offsets[j]:self.offsets[j + 1]] = synth.make_x(spec, 1000 * rank + k)
+        self.x_host = torch.from_numpy(xs).pin_memory()
+        self.x_dev = self.x_host.to(device)
+        self.y_dev = torch.zeros(self.y_offsets[-1], dtype=torch.float32, device=device)
+        self.y_host = torch.zeros(self.y_offsets[-1], dtype=torch.float32).pin_memory()
+        self.stream = torch.cuda.Stream(device=device)
+        self.graphs = []
+        self.gemv_graph = None
+
+    def xv(self, k, j):
+        return self.x_dev[k, self.offsets[j]:self.offsets[j + 1]]
+
+    def yv(self, j):
+        return self.y_dev[self.y_offsets[j]:self.y_offsets[j + 1]]
+
+    def launch_step(self, k, stream):
+        for j, lin in enumerate(self.layers):
+            lin.assign(self.xv(k, j), self.thetas[j], stream=stream)
+            lin.gemv(self.yv(j), stream=stream)
+
+    def launch_gemvs(self, stream):
+        for j, lin in enumerate(self.layers):
+            lin.gemv(self.yv(j), stream=stream)
+
+    def capture(self):
+        torch = self.torch
+        with torch.cuda.stream(self.stream):
+            for k in range(N_POOL):  # eager warm-up of every launch once
+                self.launch_step(k, self.stream)
+        self.stream.synchronize()
+        for k in range(N_POOL):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=self.stream):
+                self.launch_step(k, self.stream)
+            self.graphs.append(g)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=self.stream):
+            self.launch_gemvs(self.stream)
+        self.gemv_graph = g
+        torch.cuda.synchronize(self.device)
+
+    def bytes_per_pool_entry(self, include_x=True):
+        """Algorithmic bytes of one step for each pool entry (needs b on the host)."""
+        torch = self.torch
+        out = []
+        for k in range(N_POOL):
+            self.graphs[k].replay()
+            torch.cuda.synchronize(self.device)
+            tot = 0
+            for lin, spec in zip(self.layers, self.specs):
+                tot += min_bytes(lin.b.cpu().numpy(), spec.d_out, include_x)
+            out.append(tot)
+        return out
+
+    def effective_bits(self, k):
+        torch = self.torch
+        self.graphs[k].replay()
+        torch.cuda.synchronize(self.device)
+        return [float(lin.b.float().mean().item()) for lin in self.layers]
+
+
+def device_time_ms(torch, stream, fn, n):
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(n):
+        fn(i)
+    e1.record(stream)
+    e1.synchronize()
+    return e0.elapsed_time(e1)
+
+
+def cold_case_times(wl, reps=20):
+    """Per-GEMV device time with a cold L2: a 256 MB write before every launch."""
+    torch = wl.torch
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=wl.device)
+    rows = []
+    st = wl.stream
+    with torch.cuda.stream(st):
+        for j, (lin, spec) in enumerate(zip(wl.layers[:16], wl.specs[:16])):
+            t_all, t_gemv = [], []
+            for r in range(reps):
+                k = r % N_POOL
+                for mode in ("all", "gemv"):
+                    flush.fill_(float(r))
+                    if mode == "gemv":
+                        lin.assign(wl.xv(k, j), wl.thetas[j], stream=st)
+                        flush.fill_(float(r) + 0.5)
+                    e0 = torch.cuda.Event(enable_timing=True)
+                    e1 = torch.cuda.Event(enable_timing=True)
+                    e0.record(st)
+                    if mode == "all":
+                        lin.assign(wl.xv(k, j), wl.thetas[j], stream=st)
+                    lin.gemv(wl.yv(j), stream=st)
+                    e1.record(st)
+                    e1.synchronize()
+                    (t_all if mode == "all" else t_gemv).append(e0.elapsed_time(e1) * 1e3)
+            b = lin.b.cpu().numpy()
+            rows.append({"name": spec.name, "d_in": spec.d_in, "d_out": spec.d_out,
+                         "b_max": spec.b_max, "eff_bits": round(float(b.mean()), 3),
+                         "us_assign_gemv": round(statistics.median(t_all), 2),
+                         "us_gemv": round(statistics.median(t_gemv), 2),
+                         "gemv_GBps": round(min_bytes(b, spec.d_out, False)
+                                            / (statistics.median(t_gemv) * 1e3), 1)})
+    return rows
+
+
+def dense4_times(wl, reps=20):
+    """The in-library dense 4-bit comparator on each distinct shape, cold L2."""
+    torch = wl.torch
+    from input_adaptive_bit_b200.layer import Dense4Linear
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=wl.device)
+    seen, rows = set(), []
+    st = wl.stream
+    for j, spec in enumerate(wl.specs[:16]):
+        if (spec.d_in, spec.d_out) in seen:
+            continue
+        seen.add((spec.d_in, spec.d_out))
+        g = synth.rng(spec.config_id, 5000 + j, 0)
+        q4, s, z = synth.rtn_quantize(synth.gaussian_weights(g, spec.d_in, spec.d_out), 4)
+        d4 = Dense4Linear(q4, s, z, device=wl.device)
+        ts = []
+        with torch.cuda.stream(st):
+            for r in range(reps):
+                flush.fill_(float(r))
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record(st)
+                d4(wl.xv(r % N_POOL, j), stream=st)
+                e1.record(st)
+                e1.synchronize()
+                ts.append(e0.elapsed_time(e1) * 1e3)
+        t = statistics.median(ts)
+        nbytes = spec.d_in * spec.d_out // 2 + 4 * spec.d_out * (spec.d_in // 128) + 4 * spec.d_out
+        rows.append({"name": f"dense4_{spec.d_in}x{spec.d_out}", "us": round(t, 2),
+                     "GBps": round(nbytes / (t * 1e3), 1)})
+        del d4
+    return rows
+
+
+# ---- the oracle on the host cores (baseline only) --------------------------------
+
+def oracle_sample_run(spec, rank=0, seconds=10.0, outs_per_rep=None):
+    """Times the oracle's assign + lists + gemv on one linear of the workload.
+    Returns (GB/s-equivalent, threads, description)."""
+    import oracle
+    case = synth.make_case(spec)
+    planes = oracle.pack(case.q, spec.b_max)  # offline step, not timed
+    threads = oracle.max_threads()
+    n_out = spec.d_out if outs_per_rep is None else outs_per_rep
+    outs = None if outs_per_rep is None else np.arange(n_out, dtype=np.int32)
+    t0 = time.perf_counter()
+    reps, moved = 0, 0
+    while True:
+        b = oracle.assign(case.x, case.theta, spec.b_max)
+        oracle.lists(b, spec.b_max)
+        oracle.gemv(planes, case.s, case.z, case.x, b, spec.b_max, outs=outs, threads=threads)
+        reps += 1
+        moved += min_bytes(b, spec.d_out) * n_out / spec.d_out
+        if time.perf_counter() - t0 >= seconds:
+            break
+    dt = time.perf_counter() - t0
+    desc = (f"oracle assign+lists+gemv on {spec.name} ({spec.d_in}->{spec.d_out}), "
+            f"{n_out} outputs per run, {reps} runs in {dt:.1f} s, OpenMP over outputs")
+    return moved / dt / 1e9, threads, desc
+
+
+# ---- main ------------------------------------------------------------------------------
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    specs = workload_specs(args.workload)
+    spec = min(specs, key=lambda s: s.d_in * s.d_out)
+    # the whole run stays near two minutes whatever K and W are; every step does
+    # at least one full sample
+    budget = min(20.0, 120.0 / max(1, args.steps + args.warmup))
+    vals = []
+    for _ in range(args.warmup):
+        oracle_sample_run(spec, seconds=budget / 4, outs_per_rep=512)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        v, threads, desc = oracle_sample_run(spec, seconds=budget, outs_per_rep=512)
+        vals.append(v)
+    dt = time.perf_counter() - t0
+    value = float(np.mean(vals)) if vals else 0.0
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": UNIT,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(1e3 * dt / max(1, args.steps), 1), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": args.workload, "sampled_linear": spec.name},
+            "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": threads,
+                             "kind": "oracle", "sample": desc},
+            "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    rank, world, local = dist_env()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        dist = None
+        torch.cuda.set_device(0)
+    device = torch.device("cuda", torch.cuda.current_device())
+
+    from input_adaptive_bit_b200 import lib
+    lib()  # fail loudly if the CUDA library is missing
+
+    specs = workload_specs(args.workload)
+    wl = Workload(specs, device, rank)
+    wl.capture()
+    step_bytes = wl.bytes_per_pool_entry(include_x=True)
+    gemv_bytes = wl.bytes_per_pool_entry(include_x=False)
+    eff_bits = wl.effective_bits(0)
+
+    props = torch.cuda.get_device_properties(device)
+    gpu_id = None
+    try:
+        gpu_id = "GPU-" + str(props.uuid)
+    except Exception:
+        gpu_id = None
+    sampler = ClockSampler(gpu_id)
+
+    def barrier():
+        torch.cuda.synchronize(device)
+        if dist is not None:
+            dist.barrier()
+
+    def max_over_ranks(v):
+        if dist is None:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    # warm-up
+    with torch.cuda.stream(wl.stream):
+        for i in range(args.warmup):
+            wl.graphs[i % N_POOL].replay()
+    barrier()
+
+    # ---- timed region: K steps --------------------------------------------------
+    sampler.start()
+    time.sleep(0.3)
+    barrier()
+    with torch.cuda.stream(wl.stream):
+        ms = device_time_ms(torch, wl.stream, lambda i: wl.graphs[i % N_POOL].replay(), args.steps)
+    barrier()
+    time.sleep(0.1)
+    clocks = ClockSampler.summarize(sampler.stop())
+    ms = max_over_ranks(ms)
+    bytes_timed = sum(step_bytes[i % N_POOL] for i in range(args.steps))
+    value = world * bytes_timed / (ms * 1e-3) / 1e9
+    n_gemv = len(specs)
+
+    # ---- the dominant kernel alone: grinqh_gemv over the same 12 layers ---------
+    reps = max(20, min(2000, args.steps))
+    with torch.cuda.stream(wl.stream):
+        wl.graphs[0].replay()
+        ms_g = device_time_ms(torch, wl.stream, lambda i: wl.gemv_graph.replay(), reps)
+    ms_g = max_over_ranks(ms_g)
+    gemv_launch_us = ms_g * 1e3 / (reps * n_gemv)
+    gemv_bytes_launch = gemv_bytes[0] / n_gemv
+    peak, peak_kind = measured_peaks()
+    achieved = gemv_bytes_launch / (gemv_launch_us * 1e-6) / 1e9
+
+    # ---- end to end through the public API with host buffers --------------------
+    k_e2e = max(10, min(args.steps, 500))
+    xbytes = wl.x_host[0].numel() * 2
+    ybytes = wl.y_host.numel() * 4
+
+    def e2e_step(i):
+        k = i % N_POOL
+        wl.x_dev[k].copy_(wl.x_host[k], non_blocking=True)
+        wl.graphs[k].replay()
+        wl.y_host.copy_(wl.y_dev, non_blocking=True)
+        wl.stream.synchronize()
+
+    barrier()
+    with torch.cuda.stream(wl.stream):
+        for i in range(3):
+            e2e_step(i)
+        t0 = time.perf_counter()
+        ms_e2e = device_time_ms(torch, wl.stream, e2e_step, k_e2e)
+        wall_e2e = (time.perf_counter() - t0) * 1e3
+    ms_e2e = max_over_ranks(max(ms_e2e, wall_e2e))
+    e2e_bytes = sum(step_bytes[i % N_POOL] for i in range(k_e2e))
+    e2e_value = world * e2e_bytes / (ms_e2e * 1e-3) / 1e9
+
+    cases = None
+    dense4 = None
+    if not args.no_cases and rank == 0:
+        cases = cold_case_times(wl)
+        dense4 = dense4_times(wl)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        spec = next(s for s in specs if s.d_in * s.d_out == min(x.d_in * x.d_out for x in specs))
+        v, threads, desc = oracle_sample_run(spec, seconds=10.0)
+        cpu = {"value": round(v, 4), "unit": UNIT, "cores": threads, "kind": "oracle",
+               "sample": desc}
+
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": args.workload if args.workload != "qwen3-8b-proj"
+                   else "qwen3-8b projections at batch 1 (q 4096x4096, gate/up 4096x12288, "
+                        "down 12288x4096) x {2.0, 3.0, 4.0} effective bits, b_max 8",
+                   "gemvs_per_step": n_gemv, "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2: each step reads ~%d MB of planes from %d MB of "
+                         "distinct packed weights; no flush" % (
+                             gemv_bytes[0] // 2**20,
+                             sum(l.planes.numel() * 4 for l in wl.layers) // 2**20),
+                   "eff_bits": [round(e, 3) for e in eff_bits],
+                   "us_per_gemv": round(ms * 1e3 / (args.steps * n_gemv), 3),
+                   "bytes_per_step": int(np.mean(step_bytes))},
+        "roofline": {"bound": "hbm", "kernel": "grinqh_gemv", "achieved": round(achieved, 1),
+                     "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "traffic": None,
+                     "bytes_per_launch": int(gemv_bytes_launch),
+                     "us_per_launch": round(gemv_launch_us, 3)},
+        "e2e": {"value": round(e2e_value, 1), "unit": UNIT, "h2d_bytes_per_step": int(xbytes),
+                "d2h_bytes_per_step": int(ybytes), "steps": k_e2e,
+                "how": "pinned x H2D + step graph of the library calls + y D2H + host sync, "
+                       "every step"},
+        "gpu_launches": 2 * n_gemv * args.steps,
+        "clocks": clocks,
+        "cpu_baseline": cpu,
+    }
+    if cases is not None:
+        line["cases"] = cases
+        line["dense4"] = dense4
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,144 @@
+/*
+ * grinqh.h -- C ABI of libgrinqh, the B200 (sm_100a) batch-1 decode path of
+ * GRINQH ("Graded Input-Based Quantization Hierarchy for Efficient LLM
+ * Generation"): activation-graded precision assignment, bit-plane-sparse
+ * weight loading, on-chip reconstruction with midpoint bias correction, and
+ * the GEMV y = W_hat^T x.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Every pointer is a DEVICE pointer owned by the caller.  The library never
+ *    allocates, frees or keeps device memory between calls.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t passed as void*;
+ *    NULL means the legacy default stream).  No call synchronises with the
+ *    host, so they may be captured in a CUDA graph.
+ *  - fp16 values (x, s, z) are passed as their IEEE binary16 bit patterns.
+ *  - The return value is a status code (below).  On failure nothing has been
+ *    launched, except for GRINQH_ERR_CUDA (a launch failed); a message for the
+ *    calling thread is available from grinqh_last_error().
+ *  - Shapes: d_in % 128 == 0, 128 <= d_in <= 2^24; d_out % 16 == 0,
+ *    16 <= d_out <= 2^24; b_max in {2, 4, 6, 8}.  P = b_max/2 planes,
+ *    G = d_in/128 groups.
+ *  - Row index = input channel i (reduction dimension), output index o.
+ *
+ * Layouts (the GRINQH notes, "Key design 2": 2-bit slices stacked from most
+ * to least significant, rows stored reduction-dimension major, 16 slices per
+ * 32-bit word):
+ *    planes  uint32 [d_in][P][d_out/16]; word j of region (i, p) holds the
+ *            p-th most significant 2-bit slice of codes q[i][16j .. 16j+15],
+ *            output 16j+t in bits [2t+1 : 2t].  A row read at bit width b is
+ *            the contiguous prefix of its first b/2 regions.
+ *    s, z    fp16 [G][d_out]: scale and additive zero per (128-row group,
+ *            output channel).
+ */
+#ifndef GRINQH_H
+#define GRINQH_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes --------------------------------------------------------- */
+#define GRINQH_OK 0
+#define GRINQH_ERR_INVALID_ARG (-1)       /* null pointer, bad b_max, bad value */
+#define GRINQH_ERR_UNSUPPORTED_SHAPE (-2) /* d_in / d_out outside the rules above */
+#define GRINQH_ERR_WORKSPACE_TOO_SMALL (-3)
+#define GRINQH_ERR_CUDA (-4)              /* a CUDA runtime call or launch failed */
+#define GRINQH_ERR_DEVICE (-5)            /* a device-side check set the error word */
+
+/* Library version, major * 1000 + minor. */
+int grinqh_version(void);
+
+/* Message describing the last failing call made by this host thread ("" if
+ * none).  The pointer stays valid until the thread's next library call. */
+const char *grinqh_last_error(void);
+
+/* Bytes of device workspace that grinqh_assign + grinqh_gemv need for one
+ * (d_in, d_out, b_max) linear layer; 0 for an unsupported shape.  The
+ * workspace carries the compacted unit stream from assign to gemv, the
+ * split-K partial sums, the split-K arrival counters and a device error word.
+ * It MUST be zero-filled once after allocation (e.g. cudaMemsetAsync); every
+ * call leaves the counters and the error word back at zero.  One workspace
+ * may serve several layers in sequence on one stream (size it for the
+ * largest), but calls that overlap in time need distinct workspaces. */
+size_t grinqh_workspace_bytes(int d_in, int d_out, int b_max);
+
+/* Offline bit-plane packing ("Key design 2").
+ *   q       uint8 [d_in][d_out], codes of the b_max-bit base quantizer
+ *           (values >= 2^b_max set the device error word; their bits above
+ *           b_max are ignored).
+ *   planes  uint32 [d_in][P][d_out/16] out, layout above.
+ * Deterministic; one kernel. */
+int grinqh_pack(const uint8_t *q, int d_in, int d_out, int b_max, uint32_t *planes,
+                void *stream);
+
+/* Inverse of grinqh_pack (a test and inspection aid): q_out = codes. */
+int grinqh_unpack(const uint32_t *planes, int d_in, int d_out, int b_max, uint8_t *q_out,
+                  void *stream);
+
+/* Runtime precision assignment and row compaction ("Key design 1").
+ *   x        fp16 [d_in] decode-time input vector.
+ *   theta    fp32 [P] thresholds theta_1..theta_P (meant to be increasing):
+ *            b_i = 2 * #{k : theta_k <= |x_i|}, compared in fp32 on the
+ *            exactly converted |x_i|.  So a tie takes the higher level, -0 has
+ *            |x| = 0, +-Inf gets b_max and NaN gets b = 0.
+ *   phi      fp32 [P+1] midpoint offsets per level k (width 2k), or NULL for
+ *            the default of "Key design 3": phi_k = 2^(b_max-2k-1) for
+ *            2k < b_max and 0 at full width (nothing is truncated there).
+ *            phi[0] is never used.
+ *   b        uint8 [d_in] out: bit width of each input channel.
+ *   lists    int32 [P][d_in] out: list p holds, ascending, every i with
+ *            b_i > 2p (rows whose p-th plane is read); entries past
+ *            counts[p] are left untouched.
+ *   counts   int32 [P] out: lengths of the lists.
+ *   grp_sums fp32 [2][G] out: X_g = sum of x_i and Phi_g = sum of
+ *            x_i * phi_{b_i/2} over rows of group g with b_i > 0.
+ *   ws       workspace of grinqh_workspace_bytes(d_in, d_out, b_max) bytes
+ *            for the d_out of the grinqh_gemv that follows; assign writes
+ *            the group-ordered unit stream there.
+ * b, lists and counts are bit-exact functions of (x, theta); grp_sums are
+ * sums in a fixed order (deterministic). */
+int grinqh_assign(const uint16_t *x, const float *theta, int d_in, int b_max, const float *phi,
+                  uint8_t *b, int32_t *lists, int32_t *counts, float *grp_sums, void *ws,
+                  size_t ws_bytes, void *stream);
+
+/* The fused plane-sparse reconstruct-and-GEMV (GRINQH notes, "Method /
+ * overall framework" stages 2-3 and the custom GEMV operator):
+ *   y_o = sum over i with b_i > 0 of x_i * w_hat(i, o),
+ *   w_hat(i, o) = s[g][o] * (Q(i, o) + phi_{b_i/2}) + z[g][o],  g = i/128,
+ * where Q is the code with its low b_max - b_i bits cleared, rebuilt from the
+ * first b_i/2 planes only (the others, and every plane of a b_i = 0 row, are
+ * never read).  Consumes the unit stream that grinqh_assign left in `ws`
+ * (same d_in, b_max; the workspace must be sized for this d_out) and its
+ * grp_sums.  Writes every y[o] (fp32 [d_out]); no pre-zeroing needed.
+ * Deterministic (fixed-order split-K reduction). */
+int grinqh_gemv(const uint32_t *planes, const uint16_t *s, const uint16_t *z,
+                const float *grp_sums, int d_in, int d_out, int b_max, float *y, void *ws,
+                size_t ws_bytes, void *stream);
+
+/* Reads and clears the device error word of `ws` (synchronises `stream`).
+ * Returns GRINQH_OK, or GRINQH_ERR_DEVICE with the device code in
+ * grinqh_last_error(). */
+int grinqh_check_device_error(void *ws, void *stream);
+
+/* ---- Dense 4-bit comparator (not a GRINQH step) ------------------------------
+ * The fixed-width baseline of the GRINQH notes' throughput table ("4-bit
+ * MARLIN"), rebuilt here on the same shape, group size and fp16 s/z so the
+ * two kernels can be timed side by side.
+ *   w4 uint32 [d_in][d_out/8]: word j of row i holds 4-bit codes of outputs
+ *      8j..8j+7, output 8j+t in bits [4t+3 : 4t].
+ *   y_o = sum_i x_i * (s[g][o] * q4(i, o) + z[g][o]).  */
+int grinqh_pack_dense4(const uint8_t *q4, int d_in, int d_out, uint32_t *w4, void *stream);
+size_t grinqh_dense4_workspace_bytes(int d_in, int d_out);
+int grinqh_gemv_dense4(const uint32_t *w4, const uint16_t *s, const uint16_t *z,
+                       const uint16_t *x, int d_in, int d_out, float *y, void *ws,
+                       size_t ws_bytes, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GRINQH_H */

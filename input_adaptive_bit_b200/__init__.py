@@ -1,0 +1,145 @@
+"""Python binding of libgrinqh (argument marshalling only).
+
+Each function has the name and argument order of the C entry point in
+``include/grinqh.h``.  Array arguments may be torch tensors on the GPU (their
+``data_ptr()`` is passed) or raw integer device addresses; ``stream`` defaults
+to torch's current CUDA stream.  A non-zero status raises ``GrinqhError``.
+
+Every step of the decode path runs in the library's CUDA kernels; this module
+never computes anything itself.  If ``libgrinqh.so`` is missing or cannot be
+loaded, importing the entry points raises -- there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+__all__ = [
+    "GrinqhError", "lib", "lib_path", "grinqh_version", "grinqh_last_error",
+    "grinqh_workspace_bytes", "grinqh_pack", "grinqh_unpack", "grinqh_assign", "grinqh_gemv",
+    "grinqh_check_device_error", "grinqh_pack_dense4", "grinqh_dense4_workspace_bytes",
+    "grinqh_gemv_dense4", "EXPORTS",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+lib_path = os.path.join(_HERE, "libgrinqh.so")
+
+OK = 0
+ERR_INVALID_ARG = -1
+ERR_UNSUPPORTED_SHAPE = -2
+ERR_WORKSPACE_TOO_SMALL = -3
+ERR_CUDA = -4
+ERR_DEVICE = -5
+
+# name -> (restype, argtypes); p = pointer (passed as c_void_p), i = int, z = size_t
+_P, _I, _Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+EXPORTS = {
+    "grinqh_version": (_I, []),
+    "grinqh_last_error": (ctypes.c_char_p, []),
+    "grinqh_workspace_bytes": (_Z, [_I, _I, _I]),
+    "grinqh_pack": (_I, [_P, _I, _I, _I, _P, _P]),
+    "grinqh_unpack": (_I, [_P, _I, _I, _I, _P, _P]),
+    "grinqh_assign": (_I, [_P, _P, _I, _I, _P, _P, _P, _P, _P, _P, _Z, _P]),
+    "grinqh_gemv": (_I, [_P, _P, _P, _P, _I, _I, _I, _P, _P, _Z, _P]),
+    "grinqh_check_device_error": (_I, [_P, _P]),
+    "grinqh_pack_dense4": (_I, [_P, _I, _I, _P, _P]),
+    "grinqh_dense4_workspace_bytes": (_Z, [_I, _I]),
+    "grinqh_gemv_dense4": (_I, [_P, _P, _P, _P, _I, _I, _P, _P, _Z, _P]),
+}
+
+
+class GrinqhError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"libgrinqh status {status}: {message}")
+        self.status = status
+
+
+_lib = None
+
+
+def lib():
+    """The loaded libgrinqh (ctypes.CDLL); raises if it is not built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(lib_path):
+            raise ImportError(
+                f"{lib_path} is missing: build it with `python -m input_adaptive_bit_b200.build` "
+                "(there is no CPU fallback)")
+        handle = ctypes.CDLL(lib_path)
+        for name, (res, args) in EXPORTS.items():
+            fn = getattr(handle, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = handle
+    return _lib
+
+
+def _ptr(a):
+    if a is None:
+        return None
+    if isinstance(a, int):
+        return a
+    return a.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(status: int):
+    if status != OK:
+        raise GrinqhError(status, lib().grinqh_last_error().decode())
+
+
+def grinqh_version() -> int:
+    return lib().grinqh_version()
+
+
+def grinqh_last_error() -> str:
+    return lib().grinqh_last_error().decode()
+
+
+def grinqh_workspace_bytes(d_in: int, d_out: int, b_max: int) -> int:
+    return lib().grinqh_workspace_bytes(d_in, d_out, b_max)
+
+
+def grinqh_dense4_workspace_bytes(d_in: int, d_out: int) -> int:
+    return lib().grinqh_dense4_workspace_bytes(d_in, d_out)
+
+
+def grinqh_pack(q, d_in, d_out, b_max, planes, stream=None):
+    _check(lib().grinqh_pack(_ptr(q), d_in, d_out, b_max, _ptr(planes), _stream(stream)))
+
+
+def grinqh_unpack(planes, d_in, d_out, b_max, q_out, stream=None):
+    _check(lib().grinqh_unpack(_ptr(planes), d_in, d_out, b_max, _ptr(q_out), _stream(stream)))
+
+
+def grinqh_assign(x, theta, d_in, b_max, phi, b, lists, counts, grp_sums, ws, ws_bytes,
+                  stream=None):
+    _check(lib().grinqh_assign(_ptr(x), _ptr(theta), d_in, b_max, _ptr(phi), _ptr(b),
+                               _ptr(lists), _ptr(counts), _ptr(grp_sums), _ptr(ws), ws_bytes,
+                               _stream(stream)))
+
+
+def grinqh_gemv(planes, s, z, grp_sums, d_in, d_out, b_max, y, ws, ws_bytes, stream=None):
+    _check(lib().grinqh_gemv(_ptr(planes), _ptr(s), _ptr(z), _ptr(grp_sums), d_in, d_out,
+                             b_max, _ptr(y), _ptr(ws), ws_bytes, _stream(stream)))
+
+
+def grinqh_check_device_error(ws, stream=None):
+    _check(lib().grinqh_check_device_error(_ptr(ws), _stream(stream)))
+
+
+def grinqh_pack_dense4(q4, d_in, d_out, w4, stream=None):
+    _check(lib().grinqh_pack_dense4(_ptr(q4), d_in, d_out, _ptr(w4), _stream(stream)))
+
+
+def grinqh_gemv_dense4(w4, s, z, x, d_in, d_out, y, ws, ws_bytes, stream=None):
+    _check(lib().grinqh_gemv_dense4(_ptr(w4), _ptr(s), _ptr(z), _ptr(x), d_in, d_out, _ptr(y),
+                                    _ptr(ws), ws_bytes, _stream(stream)))

@@ -1,0 +1,88 @@
+"""Device-memory holder for one GRINQH linear layer (PyTorch plumbing only).
+
+``GrinqhLinear`` packs the layer's base codes once with ``grinqh_pack`` and
+keeps the buffers that ``grinqh_assign`` and ``grinqh_gemv`` write, so a
+decode step is two library calls on caller-owned memory.  torch allocates the
+memory and provides the stream; all arithmetic runs in libgrinqh.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import (grinqh_assign, grinqh_gemv, grinqh_gemv_dense4, grinqh_pack,
+               grinqh_pack_dense4, grinqh_dense4_workspace_bytes, grinqh_workspace_bytes)
+
+GROUP = 128
+
+
+def _dev(t, device, dtype):
+    t = torch.as_tensor(t)
+    if t.dtype != dtype:
+        raise TypeError(f"expected {dtype}, got {t.dtype}")
+    return t.to(device=device).contiguous()
+
+
+class GrinqhLinear:
+    """One decode GEMV y = W_hat^T x of GRINQH.
+
+    q: uint8 [d_in, d_out] base codes (< 2^b_max); s, z: fp16 [d_in/128, d_out].
+    """
+
+    def __init__(self, q, s, z, b_max: int, device="cuda", stream=None):
+        self.device = torch.device(device)
+        q = _dev(q, self.device, torch.uint8)
+        self.d_in, self.d_out = int(q.shape[0]), int(q.shape[1])
+        self.b_max = int(b_max)
+        self.P = self.b_max // 2
+        self.G = self.d_in // GROUP
+        self.s = _dev(s, self.device, torch.float16)
+        self.z = _dev(z, self.device, torch.float16)
+        self.planes = torch.empty((self.d_in, self.P, self.d_out // 16), dtype=torch.int32,
+                                  device=self.device)
+        grinqh_pack(q, self.d_in, self.d_out, self.b_max, self.planes, stream)
+        del q
+        # per-call buffers
+        self.b = torch.empty(self.d_in, dtype=torch.uint8, device=self.device)
+        self.lists = torch.empty((self.P, self.d_in), dtype=torch.int32, device=self.device)
+        self.counts = torch.empty(self.P, dtype=torch.int32, device=self.device)
+        self.grp_sums = torch.empty((2, self.G), dtype=torch.float32, device=self.device)
+        self.ws_bytes = grinqh_workspace_bytes(self.d_in, self.d_out, self.b_max)
+        self.ws = torch.zeros(self.ws_bytes, dtype=torch.uint8, device=self.device)
+        self.y = torch.empty(self.d_out, dtype=torch.float32, device=self.device)
+
+    def assign(self, x, theta, phi=None, stream=None):
+        grinqh_assign(x, theta, self.d_in, self.b_max, phi, self.b, self.lists, self.counts,
+                      self.grp_sums, self.ws, self.ws_bytes, stream)
+
+    def gemv(self, y=None, stream=None):
+        y = self.y if y is None else y
+        grinqh_gemv(self.planes, self.s, self.z, self.grp_sums, self.d_in, self.d_out,
+                    self.b_max, y, self.ws, self.ws_bytes, stream)
+        return y
+
+    def __call__(self, x, theta, phi=None, y=None, stream=None):
+        """x: fp16 [d_in] on the device; theta: fp32 [b_max/2] on the device."""
+        self.assign(x, theta, phi, stream)
+        return self.gemv(y, stream)
+
+
+class Dense4Linear:
+    """The in-library dense 4-bit comparator on the same shape."""
+
+    def __init__(self, q4, s, z, device="cuda", stream=None):
+        self.device = torch.device(device)
+        q4 = _dev(q4, self.device, torch.uint8)
+        self.d_in, self.d_out = int(q4.shape[0]), int(q4.shape[1])
+        self.s = _dev(s, self.device, torch.float16)
+        self.z = _dev(z, self.device, torch.float16)
+        self.w4 = torch.empty((self.d_in, self.d_out // 8), dtype=torch.int32, device=self.device)
+        grinqh_pack_dense4(q4, self.d_in, self.d_out, self.w4, stream)
+        self.ws_bytes = grinqh_dense4_workspace_bytes(self.d_in, self.d_out)
+        self.ws = torch.zeros(max(self.ws_bytes, 256), dtype=torch.uint8, device=self.device)
+        self.y = torch.empty(self.d_out, dtype=torch.float32, device=self.device)
+
+    def __call__(self, x, y=None, stream=None):
+        y = self.y if y is None else y
+        grinqh_gemv_dense4(self.w4, self.s, self.z, x, self.d_in, self.d_out, y, self.ws,
+                           self.ws_bytes, stream)
+        return y
