@@ -61,6 +61,10 @@ __global__ void __launch_bounds__(kAssignThreads) assign_kernel(AssignArgs a) {
   __shared__ int s_gcnt[kWarps][4];     // per-warp (group) counts per plane
   const int P = a.P;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // x may be written by the kernel launched just before (the previous layer):
+  // wait for it, then let the GEMV that consumes our outputs launch early.
+  asm volatile("griddepcontrol.wait;\n" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
 
   float th[4], phi[5];
 #pragma unroll
@@ -218,8 +222,17 @@ cudaError_t launch_assign(const uint16_t *x, const float *theta, int d_in, int b
   a.hdr = reinterpret_cast<WsHeader *>(ws);
   a.unit_code = reinterpret_cast<int32_t *>(static_cast<char *>(ws) + L.unit_code);
   a.unit_x = reinterpret_cast<float *>(static_cast<char *>(ws) + L.unit_x);
-  const int grid = (d_in + kAssignChunk - 1) / kAssignChunk;
-  assign_kernel<<<grid, kAssignThreads, 0, st>>>(a);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((d_in + kAssignChunk - 1) / kAssignChunk);
+  cfg.blockDim = dim3(kAssignThreads);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, assign_kernel, a);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

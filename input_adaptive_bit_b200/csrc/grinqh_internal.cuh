@@ -18,9 +18,11 @@ constexpr int kAssignThreads = 256;    // one warp per group
 constexpr int kMaxCtaUnits = 8192;     // bound on units per gemv CTA (sets the split floor)
 constexpr int kNumSMs = 148;
 constexpr int kMaxTiles = (1 << 24) / kTileOut;  // d_out <= 2^24
+constexpr int kMaxCtas = 256;                   // gemv grid: one CTA per SM, at most this many
 
 // Device error codes written to the workspace error word.
 constexpr int kDevErrStreamMismatch = 1;  // gemv saw a unit stream of another d_in / b_max
+constexpr int kDevErrBadUnit = 2;         // a unit record outside [0, d_in) x [0, P) (skipped)
 
 // Workspace header (first 256 bytes of the workspace).
 struct WsHeader {
@@ -34,23 +36,6 @@ static_assert(sizeof(WsHeader) == 256, "header size");
 
 inline __host__ __device__ size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
-// Split-K factor of grinqh_gemv for a shape: enough CTAs to cover the GPU
-// about twice, and no CTA with more than kMaxCtaUnits units in the worst case
-// (every row at full width).
-inline int gemv_splits(int d_in, int d_out, int b_max) {
-  int P = b_max / 2;
-  int tiles = (d_out + kTileOut - 1) / kTileOut;
-  long long worst_units = (long long)d_in * P;
-  int s_floor = (int)((worst_units + kMaxCtaUnits - 1) / kMaxCtaUnits);
-  int s_fill = (2 * kNumSMs + tiles - 1) / tiles;
-  int s = s_fill > s_floor ? s_fill : s_floor;
-  int s_cap = (d_in / kGroup) * P;  // no point in more splits than (group, plane) pairs
-  if (s > s_cap) s = s_cap;
-  if (s < s_floor) s = s_floor;
-  if (s < 1) s = 1;
-  return s;
-}
-
 // Workspace layout.  The header and the split-K counters sit at fixed offsets
 // for every shape, so one workspace can serve layers of different shapes in
 // turn: the counters return to zero after every gemv, whatever its shape.
@@ -59,9 +44,9 @@ struct WsLayout {
   size_t unit_code;   // int32 [P * d_in]: row << 3 | first_of_group << 2 | plane
   size_t unit_x;      // fp32 [P * d_in]: x_row * 4^(P-1-plane)
   size_t stream_end;  // end of what grinqh_assign writes
-  size_t partials;    // fp32 [splits][d_out]
+  size_t partials;    // fp32 [kMaxCtas][2][kTileOut]: partial tile segments of gemv CTAs
   size_t total;
-  int tiles, splits;
+  int tiles;
 };
 
 inline WsLayout ws_layout(int d_in, int d_out, int b_max) {
@@ -69,13 +54,12 @@ inline WsLayout ws_layout(int d_in, int d_out, int b_max) {
   int P = b_max / 2;
   size_t n_units = (size_t)d_in * P;
   L.tiles = (d_out + kTileOut - 1) / kTileOut;
-  L.splits = gemv_splits(d_in, d_out, b_max);
   L.counters = sizeof(WsHeader);
   L.unit_code = align256(L.counters + (size_t)kMaxTiles * 4);
   L.unit_x = align256(L.unit_code + n_units * 4);
   L.stream_end = align256(L.unit_x + n_units * 4);
   L.partials = L.stream_end;
-  L.total = align256(L.partials + (L.splits > 1 ? (size_t)L.splits * d_out * 4 : 0));
+  L.total = align256(L.partials + (size_t)kMaxCtas * 2 * kTileOut * 4);
   return L;
 }
 
