@@ -8,7 +8,8 @@
  * Conventions shared by every entry point
  * ---------------------------------------
  *  - Every pointer is a DEVICE pointer owned by the caller.  The library never
- *    allocates, frees or keeps device memory between calls.
+ *    allocates, frees or keeps device memory between calls (except the fixed
+ *    scratch array of grinqh_decode_gemv_noalloc, at the end of this file).
  *  - Calls are asynchronous on `stream` (a cudaStream_t passed as void*;
  *    NULL means the legacy default stream).  No call synchronises with the
  *    host, so they may be captured in a CUDA graph.
@@ -136,6 +137,30 @@ size_t grinqh_dense4_workspace_bytes(int d_in, int d_out);
 int grinqh_gemv_dense4(const uint32_t *w4, const uint16_t *s, const uint16_t *z,
                        const uint16_t *x, int d_in, int d_out, float *y, void *ws,
                        size_t ws_bytes, void *stream);
+
+/* ---- Decode GEMV without any device allocation (no counterpart in the paper:
+ * the GRINQH notes describe no such interface) ----------------------------------
+ * For callers that cannot allocate device memory -- a host framework that owns
+ * every byte of device memory and only hands its plug-ins streams and tensors,
+ * or a latency-critical path that must never enter the allocator.  It runs
+ * grinqh_assign then grinqh_gemv, keeping the assignment, lists, group sums,
+ * unit stream and split-K scratch in a fixed array (about 2.7 MB) that the
+ * library reserves on every GPU that loads it and holds until exit; it calls
+ * no cudaMalloc/cudaFree.
+ *   planes, s, z  the packed layer (as for grinqh_gemv); x, theta, phi as for
+ *                 grinqh_assign; y fp32 [d_out] out.
+ *   Limits: d_in <= 32768 and d_out <= 32768, on top of the usual shape rules;
+ *   larger shapes return GRINQH_ERR_UNSUPPORTED_SHAPE with a message.
+ * The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture.  Every call shares the one array and leaves its
+ * contents behind (the call clears what must start at zero), so calls that
+ * overlap on the GPU -- several streams, or several host threads on one
+ * device -- race and must be serialised by the caller.  Device-side checks of
+ * this path have no error word the caller can read. */
+int grinqh_decode_gemv_noalloc(const uint32_t *planes, const uint16_t *s, const uint16_t *z,
+                               const uint16_t *x, const float *theta, const float *phi,
+                               int d_in, int d_out, int b_max, float *y, void *stream);
 
 #ifdef __cplusplus
 }

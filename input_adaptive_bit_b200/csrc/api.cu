@@ -67,6 +67,14 @@ int check_ptr(const void *p, size_t align, const char *name) {
 }  // namespace
 
 namespace grinqh {
+int record_error(int code, const char *fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_msg, sizeof g_msg, fmt, ap);
+  va_end(ap);
+  return code;
+}
+
 cudaError_t ensure_smem_attr(const void *kernel, size_t bytes) {
   // One bit per (device, kernel slot); a handful of kernels use this.
   static std::atomic<unsigned long long> done[64];

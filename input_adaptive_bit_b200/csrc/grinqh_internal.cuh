@@ -63,6 +63,9 @@ inline WsLayout ws_layout(int d_in, int d_out, int b_max) {
   return L;
 }
 
+// Sets the calling thread's message (grinqh_last_error) and returns `code`.
+int record_error(int code, const char *fmt, ...);
+
 // Raises a kernel's dynamic shared memory limit to `bytes`, once per device
 // and kernel (the attribute is per device context).
 cudaError_t ensure_smem_attr(const void *kernel, size_t bytes);
