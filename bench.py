@@ -2,7 +2,7 @@
 """Throughput of the GRINQH batch-1 decode GEMV on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload qwen3-8b-proj|uniform-sweep|70b|llama3-8b-step]
+                    [--workload qwen3-8b-proj|uniform-sweep|70b|llama3-8b-step|gate-3b]
 
 A step is one pass of the whole decode path -- grinqh_assign then
 grinqh_gemv -- over one token's inputs for every linear of the workload.  The
@@ -45,6 +45,14 @@ L2_BYTES = 126 * 1024 * 1024
 N_POOL = 8
 FALLBACK_HBM_GBS = 6650.0
 
+# DRAM bytes (read + write) per grinqh_gemv launch on the qwen3-8b-proj step,
+# from one ncu capture (profiles/grinqh_gemv_qwen3-8b-proj_launches.md), keyed
+# by the SHA-256 of the gemv source it was taken on: after any change to the
+# kernel the figure no longer applies and the bench reports null.
+NCU_TRAFFIC = {
+    "84585736bc0dc9cf2ac9f0a4738586346a63ac0a4e44acbdc753bb3917df6db4": 17150844,
+}
+
 
 def parse_args(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
@@ -53,7 +61,10 @@ def parse_args(argv=None):
     ap.add_argument("--warmup", type=int, default=100)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="qwen3-8b-proj",
-                    choices=["qwen3-8b-proj", "uniform-sweep", "70b", "llama3-8b-step"])
+                    choices=["qwen3-8b-proj", "uniform-sweep", "70b", "llama3-8b-step",
+                             "gate-3b"],
+                    help="gate-3b: the single gate_proj 4096->12288 GEMV at 3 bits of the "
+                         "qwen3-8b-proj set (a small case for profiler captures)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-cases", action="store_true", help="skip the per-GEMV cold-L2 table")
     return ap.parse_args(argv)
@@ -68,6 +79,8 @@ def workload_specs(name):
         return synth.config3()
     if name == "llama3-8b-step":
         return synth.config4()
+    if name == "gate-3b":
+        return [s for s in synth.config1() if s.name == "gate_proj@3b"]
     raise ValueError(name)
 
 
@@ -78,6 +91,20 @@ def min_bytes(b: np.ndarray, d_out: int, include_x: bool = True) -> int:
     planes = int(b.astype(np.int64).sum()) * d_out // 8
     g_act = int((b.reshape(-1, 128) > 0).any(axis=1).sum())
     return planes + 4 * d_out * g_act + (2 * d_in if include_x else 0) + 4 * d_out
+
+
+def gemv_traffic(workload: str):
+    """ncu DRAM bytes per gemv launch for this kernel source, or None."""
+    if workload != "qwen3-8b-proj":
+        return None
+    import hashlib
+    path = os.path.join(ROOT, "input_adaptive_bit_b200", "csrc", "gemv.cu")
+    try:
+        with open(path, "rb") as f:
+            digest = hashlib.sha256(f.read()).hexdigest()
+    except OSError:
+        return None
+    return NCU_TRAFFIC.get(digest)
 
 
 def measured_peaks():
@@ -531,7 +558,7 @@ def main(argv=None):
                    "bytes_per_step": int(np.mean(step_bytes))},
         "roofline": {"bound": "hbm", "kernel": "grinqh_gemv", "achieved": round(achieved, 1),
                      "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
-                     "frac": round(achieved / peak, 4), "traffic": None,
+                     "frac": round(achieved / peak, 4), "traffic": gemv_traffic(args.workload),
                      "bytes_per_launch": int(gemv_bytes_launch),
                      "us_per_launch": round(gemv_launch_us, 3)},
         "e2e": {"value": round(e2e_value, 1), "unit": UNIT, "h2d_bytes_per_step": int(xbytes),

@@ -69,8 +69,7 @@ size_t grinqh_workspace_bytes(int d_in, int d_out, int b_max);
 
 /* Offline bit-plane packing ("Key design 2").
  *   q       uint8 [d_in][d_out], codes of the b_max-bit base quantizer
- *           (values >= 2^b_max set the device error word; their bits above
- *           b_max are ignored).
+ *           (only their low b_max bits are packed; higher bits are ignored).
  *   planes  uint32 [d_in][P][d_out/16] out, layout above.
  * Deterministic; one kernel. */
 int grinqh_pack(const uint8_t *q, int d_in, int d_out, int b_max, uint32_t *planes,
