@@ -4,8 +4,10 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload qwen3-8b-proj|uniform-sweep|70b|llama3-8b-step|gate-3b]
 
-A step is one pass of the whole decode path -- grinqh_assign then
-grinqh_gemv -- over one token's inputs for every linear of the workload.  The
+A step is one pass of the whole decode path over one token's inputs for every
+linear of the workload: by default the fused grinqh_decode_gemv call per linear
+(assignment, per-plane lists, counts and group sums written, then the GEMV, in
+one kernel); with --path two, grinqh_assign then grinqh_gemv.  The
 default workload is the Qwen3-8B-shaped projection set at batch 1 (q_proj
 4096->4096, gate/up 4096->12288, down 12288->4096) at 2.0, 3.0 and 4.0
 effective bits: 12 GEMVs per step, each with its own packed weights (504 MB of
@@ -45,13 +47,15 @@ L2_BYTES = 126 * 1024 * 1024
 N_POOL = 8
 FALLBACK_HBM_GBS = 6650.0
 
-# DRAM bytes (read + write) per grinqh_gemv launch on the qwen3-8b-proj step,
-# from one ncu capture (profiles/grinqh_gemv_qwen3-8b-proj_launches.md), keyed
-# by the SHA-256 of the gemv source it was taken on: after any change to the
-# kernel the figure no longer applies and the bench reports null.
+# DRAM bytes (read + write) per launch of the dominant kernel on the
+# qwen3-8b-proj step, from one ncu capture (profiles/), keyed by the SHA-256 of
+# the kernel source it was taken on: after any change to the kernel the figure
+# no longer applies and the bench reports null.
 NCU_TRAFFIC = {
+    # gemv.cu, grinqh_gemv (profiles/grinqh_gemv_qwen3-8b-proj_launches.md)
     "84585736bc0dc9cf2ac9f0a4738586346a63ac0a4e44acbdc753bb3917df6db4": 17150844,
 }
+KERNEL_SOURCE = {"fused": "decode.cu", "two": "gemv.cu"}
 
 
 def parse_args(argv=None):
@@ -60,6 +64,8 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=3000)
     ap.add_argument("--warmup", type=int, default=100)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--path", choices=["fused", "two"], default="fused",
+                    help="fused: grinqh_decode_gemv per linear; two: grinqh_assign + grinqh_gemv")
     ap.add_argument("--workload", default="qwen3-8b-proj",
                     choices=["qwen3-8b-proj", "uniform-sweep", "70b", "llama3-8b-step",
                              "gate-3b"],
@@ -93,12 +99,12 @@ def min_bytes(b: np.ndarray, d_out: int, include_x: bool = True) -> int:
     return planes + 4 * d_out * g_act + (2 * d_in if include_x else 0) + 4 * d_out
 
 
-def gemv_traffic(workload: str):
-    """ncu DRAM bytes per gemv launch for this kernel source, or None."""
+def kernel_traffic(workload: str, path: str = "fused"):
+    """ncu DRAM bytes per launch of the dominant kernel for its current source, or None."""
     if workload != "qwen3-8b-proj":
         return None
     import hashlib
-    path = os.path.join(ROOT, "input_adaptive_bit_b200", "csrc", "gemv.cu")
+    path = os.path.join(ROOT, "input_adaptive_bit_b200", "csrc", KERNEL_SOURCE[path])
     try:
         with open(path, "rb") as f:
             digest = hashlib.sha256(f.read()).hexdigest()
@@ -182,8 +188,9 @@ class ClockSampler:
 class Workload:
     """Device-resident layers, input pools and captured step graphs."""
 
-    def __init__(self, specs, device, rank):
+    def __init__(self, specs, device, rank, path="fused"):
         import torch
+        self.path = path
         from input_adaptive_bit_b200.layer import GrinqhLinear
         self.torch = torch
         self.device = device
@@ -221,6 +228,7 @@ class Workload:
         self.stream = torch.cuda.Stream(device=device)
         self.graphs = []
         self.gemv_graph = None
+        self.two_graph = None
 
     def xv(self, k, j):
         return self.x_dev[k, self.offsets[j]:self.offsets[j + 1]]
@@ -228,10 +236,14 @@ class Workload:
     def yv(self, j):
         return self.y_dev[self.y_offsets[j]:self.y_offsets[j + 1]]
 
-    def launch_step(self, k, stream):
+    def launch_step(self, k, stream, path=None):
+        path = path or self.path
         for j, lin in enumerate(self.layers):
-            lin.assign(self.xv(k, j), self.thetas[j], stream=stream)
-            lin.gemv(self.yv(j), stream=stream)
+            if path == "fused":
+                lin.decode(self.xv(k, j), self.thetas[j], y=self.yv(j), stream=stream)
+            else:
+                lin.assign(self.xv(k, j), self.thetas[j], stream=stream)
+                lin.gemv(self.yv(j), stream=stream)
 
     def launch_gemvs(self, stream):
         for j, lin in enumerate(self.layers):
@@ -240,14 +252,20 @@ class Workload:
     def capture(self):
         torch = self.torch
         with torch.cuda.stream(self.stream):
-            for k in range(N_POOL):  # eager warm-up of every launch once
-                self.launch_step(k, self.stream)
+            for k in range(N_POOL):  # eager warm-up of every launch once, both paths
+                self.launch_step(k, self.stream, "two")
+                self.launch_step(k, self.stream, "fused")
         self.stream.synchronize()
         for k in range(N_POOL):
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=self.stream):
                 self.launch_step(k, self.stream)
             self.graphs.append(g)
+        # the two-kernel path as a comparison: a whole step, and its gemv launches alone
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=self.stream):
+            self.launch_step(0, self.stream, "two")
+        self.two_graph = g
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=self.stream):
             self.launch_gemvs(self.stream)
@@ -286,17 +304,18 @@ def device_time_ms(torch, stream, fn, n):
 
 
 def cold_case_times(wl, reps=20):
-    """Per-GEMV device time with a cold L2: a 256 MB write before every launch."""
+    """Per-GEMV device time with a cold L2 (a 256 MB write before every launch):
+    the fused decode call, assign + gemv, and gemv alone."""
     torch = wl.torch
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=wl.device)
     rows = []
     st = wl.stream
     with torch.cuda.stream(st):
         for j, (lin, spec) in enumerate(zip(wl.layers[:16], wl.specs[:16])):
-            t_all, t_gemv = [], []
+            t = {"fused": [], "all": [], "gemv": []}
             for r in range(reps):
                 k = r % N_POOL
-                for mode in ("all", "gemv"):
+                for mode in t:
                     flush.fill_(float(r))
                     if mode == "gemv":
                         lin.assign(wl.xv(k, j), wl.thetas[j], stream=st)
@@ -304,19 +323,25 @@ def cold_case_times(wl, reps=20):
                     e0 = torch.cuda.Event(enable_timing=True)
                     e1 = torch.cuda.Event(enable_timing=True)
                     e0.record(st)
-                    if mode == "all":
-                        lin.assign(wl.xv(k, j), wl.thetas[j], stream=st)
-                    lin.gemv(wl.yv(j), stream=st)
+                    if mode == "fused":
+                        lin.decode(wl.xv(k, j), wl.thetas[j], y=wl.yv(j), stream=st)
+                    else:
+                        if mode == "all":
+                            lin.assign(wl.xv(k, j), wl.thetas[j], stream=st)
+                        lin.gemv(wl.yv(j), stream=st)
                     e1.record(st)
                     e1.synchronize()
-                    (t_all if mode == "all" else t_gemv).append(e0.elapsed_time(e1) * 1e3)
+                    t[mode].append(e0.elapsed_time(e1) * 1e3)
             b = lin.b.cpu().numpy()
+            med = {m: statistics.median(v) for m, v in t.items()}
             rows.append({"name": spec.name, "d_in": spec.d_in, "d_out": spec.d_out,
                          "b_max": spec.b_max, "eff_bits": round(float(b.mean()), 3),
-                         "us_assign_gemv": round(statistics.median(t_all), 2),
-                         "us_gemv": round(statistics.median(t_gemv), 2),
+                         "us_fused": round(med["fused"], 2),
+                         "fused_GBps": round(min_bytes(b, spec.d_out) / (med["fused"] * 1e3), 1),
+                         "us_assign_gemv": round(med["all"], 2),
+                         "us_gemv": round(med["gemv"], 2),
                          "gemv_GBps": round(min_bytes(b, spec.d_out, False)
-                                            / (statistics.median(t_gemv) * 1e3), 1)})
+                                            / (med["gemv"] * 1e3), 1)})
     return rows
 
 
@@ -442,7 +467,7 @@ def main(argv=None):
     lib()  # fail loudly if the CUDA library is missing
 
     specs = workload_specs(args.workload)
-    wl = Workload(specs, device, rank)
+    wl = Workload(specs, device, rank, args.path)
     wl.capture()
     step_bytes = wl.bytes_per_pool_entry(include_x=True)
     gemv_bytes = wl.bytes_per_pool_entry(include_x=False)
@@ -488,16 +513,31 @@ def main(argv=None):
     value = world * bytes_timed / (ms * 1e-3) / 1e9
     n_gemv = len(specs)
 
-    # ---- the dominant kernel alone: grinqh_gemv over the same 12 layers ---------
+    # ---- the dominant kernel -------------------------------------------------------
+    # fused: the step is n_gemv launches of the one decode kernel, timed above;
+    # two: grinqh_gemv alone over the same layers (after an assign of pool entry 0)
     reps = max(20, min(2000, args.steps))
     with torch.cuda.stream(wl.stream):
-        wl.graphs[0].replay()
+        wl.two_graph.replay()
         ms_g = device_time_ms(torch, wl.stream, lambda i: wl.gemv_graph.replay(), reps)
+        ms_two = device_time_ms(torch, wl.stream, lambda i: wl.two_graph.replay(), reps)
     ms_g = max_over_ranks(ms_g)
+    ms_two = max_over_ranks(ms_two)
     gemv_launch_us = ms_g * 1e3 / (reps * n_gemv)
-    gemv_bytes_launch = gemv_bytes[0] / n_gemv
     peak, peak_kind = measured_peaks()
-    achieved = gemv_bytes_launch / (gemv_launch_us * 1e-6) / 1e9
+    if args.path == "fused":
+        kernel_name = "decode_kernel (grinqh_decode_gemv)"
+        launch_us = ms * 1e3 / (args.steps * n_gemv)
+        bytes_launch = bytes_timed / (args.steps * n_gemv)
+    else:
+        kernel_name = "gemv_kernel (grinqh_gemv)"
+        launch_us = gemv_launch_us
+        bytes_launch = gemv_bytes[0] / n_gemv
+    achieved = bytes_launch / (launch_us * 1e-6) / 1e9
+    two_kernel = {"ms_per_step": round(ms_two / reps, 5),
+                  "value": round(step_bytes[0] / (ms_two / reps * 1e-3) / 1e9, 1),
+                  "gemv_us_per_launch": round(gemv_launch_us, 3),
+                  "gemv_GBps": round(gemv_bytes[0] / n_gemv / (gemv_launch_us * 1e-6) / 1e9, 1)}
 
     # ---- end to end through the public API with host buffers --------------------
     k_e2e = max(10, min(args.steps, 500))
@@ -556,16 +596,19 @@ def main(argv=None):
                    "eff_bits": [round(e, 3) for e in eff_bits],
                    "us_per_gemv": round(ms * 1e3 / (args.steps * n_gemv), 3),
                    "bytes_per_step": int(np.mean(step_bytes))},
-        "roofline": {"bound": "hbm", "kernel": "grinqh_gemv", "achieved": round(achieved, 1),
+        "roofline": {"bound": "hbm", "kernel": kernel_name, "achieved": round(achieved, 1),
                      "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
-                     "frac": round(achieved / peak, 4), "traffic": gemv_traffic(args.workload),
-                     "bytes_per_launch": int(gemv_bytes_launch),
-                     "us_per_launch": round(gemv_launch_us, 3)},
+                     "frac": round(achieved / peak, 4),
+                     "traffic": kernel_traffic(args.workload, args.path),
+                     "bytes_per_launch": int(bytes_launch),
+                     "us_per_launch": round(launch_us, 3)},
         "e2e": {"value": round(e2e_value, 1), "unit": UNIT, "h2d_bytes_per_step": int(xbytes),
                 "d2h_bytes_per_step": int(ybytes), "steps": k_e2e,
                 "how": "pinned x H2D + step graph of the library calls + y D2H + host sync, "
                        "every step"},
-        "gpu_launches": 2 * n_gemv * args.steps,
+        "gpu_launches": (1 if args.path == "fused" else 2) * n_gemv * args.steps,
+        "path": args.path,
+        "two_kernel_path": two_kernel,
         "clocks": clocks,
         "cpu_baseline": cpu,
     }

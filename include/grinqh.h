@@ -119,6 +119,30 @@ int grinqh_gemv(const uint32_t *planes, const uint16_t *s, const uint16_t *z,
                 const float *grp_sums, int d_in, int d_out, int b_max, float *y, void *ws,
                 size_t ws_bytes, void *stream);
 
+/* The whole decode step in one kernel (the GRINQH notes, "Method / overall
+ * framework" stages 1-3: grinqh_assign followed by grinqh_gemv, fused): every
+ * CTA derives the precision assignment and the per-plane compaction it needs
+ * from x and theta itself, so no unit stream goes through device memory and
+ * no second launch waits on the first.
+ *   planes, s, z  the packed layer, as for grinqh_gemv.
+ *   x, theta, phi as for grinqh_assign.
+ *   y             fp32 [d_out] out, the same value grinqh_gemv computes after
+ *                 grinqh_assign (within the rounding of a different summation
+ *                 order); every y[o] is written.
+ *   b, lists, counts, grp_sums  optional outputs with exactly the contents
+ *                 grinqh_assign writes (bit-exact, grp_sums in the same order);
+ *                 pass NULL for any of them to skip it.
+ *   ws            workspace of grinqh_workspace_bytes(d_in, d_out, b_max)
+ *                 bytes (zero-filled once; left zeroed), used for the split-K
+ *                 partial sums and counters only.
+ * Limits: d_in <= 65536 (GRINQH_ERR_UNSUPPORTED_SHAPE otherwise; use
+ * grinqh_assign + grinqh_gemv there).  Deterministic. */
+int grinqh_decode_gemv(const uint32_t *planes, const uint16_t *s, const uint16_t *z,
+                       const uint16_t *x, const float *theta, const float *phi, int d_in,
+                       int d_out, int b_max, float *y, uint8_t *b, int32_t *lists,
+                       int32_t *counts, float *grp_sums, void *ws, size_t ws_bytes,
+                       void *stream);
+
 /* Reads and clears the device error word of `ws` (synchronises `stream`).
  * Returns GRINQH_OK, or GRINQH_ERR_DEVICE with the device code in
  * grinqh_last_error(). */

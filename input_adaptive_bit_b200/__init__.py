@@ -18,7 +18,7 @@ __all__ = [
     "GrinqhError", "lib", "lib_path", "grinqh_version", "grinqh_last_error",
     "grinqh_workspace_bytes", "grinqh_pack", "grinqh_unpack", "grinqh_assign", "grinqh_gemv",
     "grinqh_check_device_error", "grinqh_pack_dense4", "grinqh_dense4_workspace_bytes",
-    "grinqh_gemv_dense4", "grinqh_decode_gemv_noalloc", "EXPORTS",
+    "grinqh_gemv_dense4", "grinqh_decode_gemv", "grinqh_decode_gemv_noalloc", "EXPORTS",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -45,6 +45,8 @@ EXPORTS = {
     "grinqh_pack_dense4": (_I, [_P, _I, _I, _P, _P]),
     "grinqh_dense4_workspace_bytes": (_Z, [_I, _I]),
     "grinqh_gemv_dense4": (_I, [_P, _P, _P, _P, _I, _I, _P, _P, _Z, _P]),
+    "grinqh_decode_gemv": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _P, _P, _P, _P, _P, _P,
+                                _Z, _P]),
     "grinqh_decode_gemv_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _P, _P]),
 }
 
@@ -144,6 +146,15 @@ def grinqh_pack_dense4(q4, d_in, d_out, w4, stream=None):
 def grinqh_gemv_dense4(w4, s, z, x, d_in, d_out, y, ws, ws_bytes, stream=None):
     _check(lib().grinqh_gemv_dense4(_ptr(w4), _ptr(s), _ptr(z), _ptr(x), d_in, d_out, _ptr(y),
                                     _ptr(ws), ws_bytes, _stream(stream)))
+
+
+def grinqh_decode_gemv(planes, s, z, x, theta, phi, d_in, d_out, b_max, y, b, lists, counts,
+                       grp_sums, ws, ws_bytes, stream=None):
+    """assign + gemv fused into one kernel; b, lists, counts, grp_sums may be None."""
+    _check(lib().grinqh_decode_gemv(_ptr(planes), _ptr(s), _ptr(z), _ptr(x), _ptr(theta),
+                                    _ptr(phi), d_in, d_out, b_max, _ptr(y), _ptr(b), _ptr(lists),
+                                    _ptr(counts), _ptr(grp_sums), _ptr(ws), ws_bytes,
+                                    _stream(stream)))
 
 
 def grinqh_decode_gemv_noalloc(planes, s, z, x, theta, phi, d_in, d_out, b_max, y, stream=None):

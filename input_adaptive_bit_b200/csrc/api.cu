@@ -176,6 +176,40 @@ int grinqh_gemv(const uint32_t *planes, const uint16_t *s, const uint16_t *z,
                      "grinqh_gemv launch");
 }
 
+int grinqh_decode_gemv(const uint32_t *planes, const uint16_t *s, const uint16_t *z,
+                       const uint16_t *x, const float *theta, const float *phi, int d_in,
+                       int d_out, int b_max, float *y, uint8_t *b, int32_t *lists,
+                       int32_t *counts, float *grp_sums, void *ws, size_t ws_bytes,
+                       void *stream) {
+  TRY(check_bmax(b_max));
+  TRY(check_din(d_in));
+  TRY(check_dout(d_out));
+  if (d_in > grinqh::kDecodeMaxDin)
+    return fail(GRINQH_ERR_UNSUPPORTED_SHAPE,
+                "grinqh_decode_gemv: d_in must be <= %d (got %d); use grinqh_assign + "
+                "grinqh_gemv",
+                grinqh::kDecodeMaxDin, d_in);
+  TRY(check_ptr(planes, (d_out / 16) % 4 == 0 ? 16 : 4, "planes"));
+  TRY(check_ptr(s, 16, "s"));
+  TRY(check_ptr(z, 16, "z"));
+  TRY(check_ptr(x, 16, "x"));
+  TRY(check_ptr(theta, 4, "theta"));
+  if (phi) TRY(check_ptr(phi, 4, "phi"));
+  TRY(check_ptr(y, 4, "y"));
+  if (lists) TRY(check_ptr(lists, 4, "lists"));
+  if (counts) TRY(check_ptr(counts, 4, "counts"));
+  if (grp_sums) TRY(check_ptr(grp_sums, 4, "grp_sums"));
+  TRY(check_ptr(ws, 256, "ws"));
+  const size_t need = grinqh::ws_layout(d_in, d_out, b_max).total;
+  if (ws_bytes < need)
+    return fail(GRINQH_ERR_WORKSPACE_TOO_SMALL, "workspace of %zu bytes, decode needs %zu",
+                ws_bytes, need);
+  return cuda_status(grinqh::launch_decode(planes, s, z, x, theta, phi, d_in, d_out, b_max, y,
+                                           b, lists, counts, grp_sums, ws,
+                                           (cudaStream_t)stream),
+                     "grinqh_decode_gemv launch");
+}
+
 int grinqh_check_device_error(void *ws, void *stream) {
   TRY(check_ptr(ws, 256, "ws"));
   int code = 0;

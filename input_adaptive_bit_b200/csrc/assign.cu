@@ -45,13 +45,6 @@ __device__ __forceinline__ int level_count(float a, const float (&th)[4], int P)
   return c;
 }
 
-__device__ __forceinline__ float pick(const float (&v)[5], int k) {
-  float r = v[0];
-#pragma unroll
-  for (int j = 1; j < 5; ++j) r = (k == j) ? v[j] : r;
-  return r;
-}
-
 __device__ __forceinline__ float half_bits_to_float(uint16_t h) {
   return __half2float(__ushort_as_half(h));
 }
@@ -111,7 +104,6 @@ __global__ void __launch_bounds__(kAssignThreads) assign_kernel(AssignArgs a) {
   float xf[4];
   int gc[4] = {0, 0, 0, 0};
   if (has_group) {
-    float xs = 0.0f, ps = 0.0f;
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
       const int i = g * kGroup + 32 * r + lane;
@@ -124,19 +116,20 @@ __global__ void __launch_bounds__(kAssignThreads) assign_kernel(AssignArgs a) {
         mask[r][p] = __ballot_sync(0xffffffffu, cnt[r] > p);
         gc[p] += __popc(mask[r][p]);
       }
-      if (cnt[r] > 0) {
-        xs += xf[r];
-        ps += xf[r] * pick(phi, cnt[r]);
-      }
     }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      xs += __shfl_xor_sync(0xffffffffu, xs, off);
-      ps += __shfl_xor_sync(0xffffffffu, ps, off);
-    }
+    // X_g, Phi_g in the fixed order of group_sums8 (16 lanes x 8 rows), the
+    // order the fused decode kernel uses too; lanes 16-31 repeat lanes 0-15
+    __half2 t2[4];
+    make_thresholds(a.theta, P, t2);
+    const uint4 xw =
+        __ldg(reinterpret_cast<const uint4 *>(a.x + g * kGroup + 8 * (lane & 15)));
+    uint32_t mk[4];
+    plane_masks8(xw, t2, P, mk);
+    float X, Phi;
+    group_sums8(xw, mk, phi, X, Phi);
     if (lane == 0) {
-      a.grp_sums[g] = xs;
-      a.grp_sums[a.G + g] = ps;
+      a.grp_sums[g] = X;
+      a.grp_sums[a.G + g] = Phi;
     }
   }
   if (lane == 0) {

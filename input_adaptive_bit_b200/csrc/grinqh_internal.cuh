@@ -19,6 +19,7 @@ constexpr int kMaxCtaUnits = 8192;     // bound on units per gemv CTA (sets the 
 constexpr int kNumSMs = 148;
 constexpr int kMaxTiles = (1 << 24) / kTileOut;  // d_out <= 2^24
 constexpr int kMaxCtas = 256;                   // gemv grid: one CTA per SM, at most this many
+constexpr int kDecodeMaxDin = 65536;            // largest d_in of the fused decode kernel
 
 // Device error codes written to the workspace error word.
 constexpr int kDevErrStreamMismatch = 1;  // gemv saw a unit stream of another d_in / b_max
@@ -63,6 +64,90 @@ inline WsLayout ws_layout(int d_in, int d_out, int b_max) {
   return L;
 }
 
+// ---- precision assignment on 8 consecutive rows (shared by assign and decode) --------
+//
+// b_i = 2 #{k : theta_k <= |x_i|}.  With the thresholds sorted ascending (NaN
+// last: a NaN threshold never counts), b_i > 2p holds exactly when the p-th
+// smallest threshold is <= |x_i|; and since |x_i| is an fp16 value, |x_i| >=
+// theta holds exactly when |x_i| >= (theta rounded up to fp16).  So one packed
+// fp16 comparison per two rows and plane gives the plane masks bit-exactly.
+
+// Sorted, fp16-rounded-up thresholds; entries past P (and NaN thresholds) are NaN.
+__device__ __forceinline__ void make_thresholds(const float *theta, int P, __half2 (&t2)[4]) {
+  float th[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) th[k] = (k < P) ? theta[k] : __int_as_float(0x7fc00000);
+  auto cs = [](float &x, float &y) {
+    const bool sw = (x != x) ? (y == y) : (y < x);
+    if (sw) {
+      const float t = x;
+      x = y;
+      y = t;
+    }
+  };
+  cs(th[0], th[1]);
+  cs(th[2], th[3]);
+  cs(th[0], th[2]);
+  cs(th[1], th[3]);
+  cs(th[1], th[2]);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) t2[k] = __half2half2(__float2half_ru(th[k]));
+}
+
+// mask[p] bit e = (row e of the 8 rows in xw has b > 2p); rows in memory order.
+__device__ __forceinline__ void plane_masks8(uint4 xw, const __half2 (&t2)[4], int P,
+                                             uint32_t (&mask)[4]) {
+  const uint32_t w[4] = {xw.x & 0x7fff7fffu, xw.y & 0x7fff7fffu, xw.z & 0x7fff7fffu,
+                         xw.w & 0x7fff7fffu};
+#pragma unroll
+  for (int p = 0; p < 4; ++p) {
+    uint32_t v = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      v |= (__hge2_mask(*reinterpret_cast<const __half2 *>(&w[j]), t2[p]) & 0x00010001u) << (2 * j);
+    mask[p] = (p < P) ? ((v | (v >> 15)) & 0xFFu) : 0u;
+  }
+}
+
+// Level (b/2) of row e from its plane masks.
+__device__ __forceinline__ int row_level(const uint32_t (&mask)[4], int e) {
+  return (int)(((mask[0] >> e) & 1u) + ((mask[1] >> e) & 1u) + ((mask[2] >> e) & 1u) +
+               ((mask[3] >> e) & 1u));
+}
+
+__device__ __forceinline__ float pick_phi(const float (&phi)[5], int k) {
+  float r = phi[0];
+#pragma unroll
+  for (int j = 1; j < 5; ++j) r = (k == j) ? phi[j] : r;
+  return r;
+}
+
+// X_g = sum of x and Phi_g = sum of x phi_{b/2} over the active rows of a
+// 128-row group held by 16 consecutive lanes (8 rows each): each lane sums its
+// rows in order, then the 16 lanes are added pairwise (xor 8, 4, 2, 1).  Every
+// lane of the warp must call it (the shuffles span the whole warp).
+__device__ __forceinline__ void group_sums8(uint4 xw, const uint32_t (&mask)[4],
+                                            const float (&phi)[5], float &X, float &Phi) {
+  const uint32_t w[4] = {xw.x, xw.y, xw.z, xw.w};
+  float xs = 0.0f, ps = 0.0f;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const int lev = row_level(mask, e);
+    const float xv = __half2float(__ushort_as_half((uint16_t)(w[e >> 1] >> (16 * (e & 1)))));
+    if (lev > 0) {
+      xs += xv;
+      ps = __fmaf_rn(xv, pick_phi(phi, lev), ps);
+    }
+  }
+#pragma unroll
+  for (int off = 8; off > 0; off >>= 1) {
+    xs += __shfl_xor_sync(0xffffffffu, xs, off);
+    ps += __shfl_xor_sync(0xffffffffu, ps, off);
+  }
+  X = xs;
+  Phi = ps;
+}
+
 // Sets the calling thread's message (grinqh_last_error) and returns `code`.
 int record_error(int code, const char *fmt, ...);
 
@@ -82,6 +167,10 @@ cudaError_t launch_assign(const uint16_t *x, const float *theta, int d_in, int b
 cudaError_t launch_gemv(const uint32_t *planes, const uint16_t *s, const uint16_t *z,
                         const float *grp_sums, int d_in, int d_out, int b_max, float *y,
                         void *ws, cudaStream_t st);
+cudaError_t launch_decode(const uint32_t *planes, const uint16_t *s, const uint16_t *z,
+                          const uint16_t *x, const float *theta, const float *phi, int d_in,
+                          int d_out, int b_max, float *y, uint8_t *b, int32_t *lists,
+                          int32_t *counts, float *grp_sums, void *ws, cudaStream_t st);
 cudaError_t launch_pack_dense4(const uint8_t *q4, int d_in, int d_out, uint32_t *w4,
                                cudaStream_t st);
 size_t dense4_ws_bytes(int d_in, int d_out);

@@ -9,7 +9,7 @@ from __future__ import annotations
 
 import torch
 
-from . import (grinqh_assign, grinqh_gemv, grinqh_gemv_dense4, grinqh_pack,
+from . import (grinqh_assign, grinqh_decode_gemv, grinqh_gemv, grinqh_gemv_dense4, grinqh_pack,
                grinqh_pack_dense4, grinqh_dense4_workspace_bytes, grinqh_workspace_bytes)
 
 GROUP = 128
@@ -58,6 +58,17 @@ class GrinqhLinear:
         y = self.y if y is None else y
         grinqh_gemv(self.planes, self.s, self.z, self.grp_sums, self.d_in, self.d_out,
                     self.b_max, y, self.ws, self.ws_bytes, stream)
+        return y
+
+    def decode(self, x, theta, phi=None, y=None, outputs=True, stream=None):
+        """The fused single-kernel decode step; with outputs=True it also fills
+        b, lists, counts and grp_sums as grinqh_assign would."""
+        y = self.y if y is None else y
+        o = outputs
+        grinqh_decode_gemv(self.planes, self.s, self.z, x, theta, phi, self.d_in, self.d_out,
+                           self.b_max, y, self.b if o else None, self.lists if o else None,
+                           self.counts if o else None, self.grp_sums if o else None, self.ws,
+                           self.ws_bytes, stream)
         return y
 
     def __call__(self, x, theta, phi=None, y=None, stream=None):

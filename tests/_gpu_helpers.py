@@ -16,15 +16,21 @@ def to_dev(a, device="cuda"):
     return torch.from_numpy(np.ascontiguousarray(a)).to(device)
 
 
-def run_layer(q, s, z, x, theta, b_max, phi=None, lin=None):
-    """Runs pack (unless `lin` is given), assign and gemv; returns host copies."""
+def run_layer(q, s, z, x, theta, b_max, phi=None, lin=None, path="two"):
+    """Runs pack (unless `lin` is given), then assign + gemv (path "two") or the
+    fused decode kernel (path "fused"); returns host copies."""
     if lin is None:
         lin = GrinqhLinear(q, s, z, b_max)
     xd = to_dev(x)
     th = to_dev(np.asarray(theta, np.float32))
     ph = None if phi is None else to_dev(np.asarray(phi, np.float32))
     lin.lists.fill_(-7)
-    y = lin(xd, th, ph)
+    if path == "two":
+        y = lin(xd, th, ph)
+    elif path == "fused":
+        y = lin.decode(xd, th, ph)
+    else:
+        raise ValueError(path)
     torch.cuda.synchronize()
     return lin, {
         "b": lin.b.cpu().numpy(),
@@ -73,12 +79,13 @@ def check_y(out, planes_ref, s, z, x, b_ref, b_max, phi=None, outs=None, threads
     return y_ref, bound
 
 
-def full_case_check(case: synth.Case, phi=None, sample_outputs=None, sample_rows=None, seed=0):
+def full_case_check(case: synth.Case, phi=None, sample_outputs=None, sample_rows=None, seed=0,
+                    path="two"):
     """Parity of one generated case.  Small cases compare everything; large ones
     compare b/lists/counts fully, planes on sampled rows and y on sampled outputs."""
     lin_spec = case.lin
     b_max = lin_spec.b_max
-    lin, out = run_layer(case.q, case.s, case.z, case.x, case.theta, b_max, phi)
+    lin, out = run_layer(case.q, case.s, case.z, case.x, case.theta, b_max, phi, path=path)
     b_ref = check_assign(out, case.x, case.theta, b_max)
     planes = planes_host(lin)
     rng = np.random.default_rng(seed)

@@ -103,6 +103,27 @@ def test_gemv_argument_checks():
     assert _status("grinqh_gemv", *bmax) == gq.ERR_INVALID_ARG
 
 
+def test_decode_argument_checks():
+    need = gq.grinqh_workspace_bytes(256, 64, 8)
+    args = [FAKE, FAKE, FAKE, FAKE, FAKE, None, 256, 64, 8, FAKE, None, None, None, None, FAKE,
+            need, None]
+    for k in (0, 1, 2, 3, 4, 9, 14):
+        bad = list(args)
+        bad[k] = None
+        assert _status("grinqh_decode_gemv", *bad) == gq.ERR_INVALID_ARG, k
+    small = list(args)
+    small[15] = need - 1
+    assert _status("grinqh_decode_gemv", *small) == gq.ERR_WORKSPACE_TOO_SMALL
+    big = list(args)
+    big[6] = 65536 + 128
+    big[15] = 1 << 40
+    assert _status("grinqh_decode_gemv", *big) == gq.ERR_UNSUPPORTED_SHAPE
+    assert "65536" in gq.grinqh_last_error()
+    unaligned_x = list(args)
+    unaligned_x[3] = FAKE + 8
+    assert _status("grinqh_decode_gemv", *unaligned_x) == gq.ERR_INVALID_ARG
+
+
 def test_dense4_argument_checks():
     need = gq.grinqh_dense4_workspace_bytes(256, 64)
     assert need > 0

@@ -1,0 +1,120 @@
+"""GPU parity of the fused decode kernel (grinqh_decode_gemv) in the cases its
+own work split creates: ranges spanning several rounds, more tiles than CTAs,
+empty groups between active ones, the largest accepted d_in, fewer units than
+CTAs, and the optional outputs (bit-exact with grinqh_assign, or skipped)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from _gpu_helpers import check_assign, check_y, run_layer, to_dev
+from input_adaptive_bit_b200.layer import GrinqhLinear
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    torch.cuda.init()
+
+
+def cheap_case(seed, d_in, d_out, b_max, fractions=None):
+    """Uniform random codes and fp16 s/z (no RTN pass), synthetic x and Theta."""
+    g = np.random.default_rng(seed)
+    P = b_max // 2
+    q = g.integers(0, 1 << b_max, size=(d_in, d_out), dtype=np.uint8)
+    s = (g.random((d_in // 128, d_out)) * 0.01 + 1e-4).astype(np.float16)
+    z = (-(g.random((d_in // 128, d_out)) * 0.5)).astype(np.float16)
+    x = synth.activations(g, d_in)
+    fr = np.full(P + 1, 1.0 / (P + 1)) if fractions is None else np.asarray(fractions)
+    theta = synth.quantile_thresholds(np.abs(x.astype(np.float32)), fr)
+    return q, s, z, x, theta
+
+
+def check_fused(q, s, z, x, theta, b_max, outs=None):
+    lin, out = run_layer(q, s, z, x, theta, b_max, path="fused")
+    b_ref = check_assign(out, x, theta, b_max)
+    check_y(out, oracle.pack(q, b_max), s, z, x, b_ref, b_max, outs=outs)
+    return lin, out
+
+
+def test_optional_outputs_match_assign_bit_for_bit_or_are_skipped():
+    q, s, z, x, theta = cheap_case(1, 2048, 3072, 8)
+    lin = GrinqhLinear(q, s, z, 8)
+    xd, th = to_dev(x), to_dev(theta)
+    lin.assign(xd, th)
+    torch.cuda.synchronize()
+    ref = {k: getattr(lin, k).clone() for k in ("b", "lists", "counts", "grp_sums")}
+    for k in ref:
+        getattr(lin, k).fill_(0)
+    y1 = lin.decode(xd, th).clone()
+    torch.cuda.synchronize()
+    assert torch.equal(lin.b, ref["b"]) and torch.equal(lin.counts, ref["counts"])
+    n = ref["counts"].cpu().numpy()
+    for p in range(4):
+        assert torch.equal(lin.lists[p, :n[p]], ref["lists"][p, :n[p]])
+    assert torch.equal(lin.grp_sums.view(torch.int32), ref["grp_sums"].view(torch.int32))
+    # outputs skipped: nothing written, y identical
+    for k in ref:
+        getattr(lin, k).fill_(-3)
+    y2 = lin.decode(xd, th, outputs=False)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2)
+    assert (lin.b == 253).all() and (lin.lists == -3).all() and (lin.counts == -3).all()
+    assert (lin.grp_sums == -3).all()
+
+
+def test_more_tiles_than_ctas_and_several_rounds_per_range():
+    # d_out = 148 * 1024 + 16: 149 tiles (one CTA takes two), the last ragged and
+    # not 16-byte aligned (d_out / 16 odd); 10 groups and ~2500 units per tile
+    # force rounds cut both by the 8-group window and by the 1024-unit cap
+    d_in, d_out = 1280, 148 * 1024 + 16
+    q, s, z, x, theta = cheap_case(2, d_in, d_out, 8)
+    outs = np.unique(np.concatenate([np.arange(0, 64), np.arange(d_out - 80, d_out),
+                                     np.random.default_rng(0).integers(0, d_out, 200)]))
+    check_fused(q, s, z, x, theta, 8, outs=outs.astype(np.int32))
+
+
+@pytest.mark.parametrize("live", [[0, 31], [0, 7, 8, 20, 31], [5], [31]])
+def test_empty_groups_between_active_ones(live):
+    d_in, d_out = 4096, 2048
+    q, s, z, x, theta = cheap_case(3, d_in, d_out, 8)
+    keep = np.zeros(d_in, bool)
+    for g in live:
+        keep[128 * g:128 * (g + 1)] = True
+    x = np.where(keep, x, np.float16(0.0)).astype(np.float16)
+    theta = np.array([1e-3, 0.5, 1.0, 2.0], np.float32)
+    check_fused(q, s, z, x, theta, 8)
+
+
+def test_largest_accepted_d_in():
+    q, s, z, x, theta = cheap_case(4, 65536, 64, 8)
+    check_fused(q, s, z, x, theta, 8)
+
+
+@pytest.mark.parametrize("n_active", [1, 3, 40])
+def test_fewer_units_than_ctas(n_active):
+    d_in, d_out = 1024, 4096
+    q, s, z, x, _ = cheap_case(5, d_in, d_out, 8)
+    g = np.random.default_rng(n_active)
+    x = (g.standard_normal(d_in) * 0.01).astype(np.float16)
+    idx = g.choice(d_in, n_active, replace=False)
+    x[idx] = (g.standard_normal(n_active) + 4.0).astype(np.float16)
+    theta = np.array([1.0, 2.0, 3.0, 100.0], np.float32)
+    check_fused(q, s, z, x, theta, 8)
+
+
+@pytest.mark.parametrize("b_max", [2, 4, 6])
+def test_smaller_base_widths_on_wide_layers(b_max):
+    q, s, z, x, theta = cheap_case(6, 2048, 5120, b_max)
+    check_fused(q, s, z, x, theta, b_max)
+
+
+def test_large_activations_use_a_scaled_b_column():
+    # |x| * 4^(P-1) beyond the fp16 range: the kernel scales each group's column
+    q, s, z, x, theta = cheap_case(7, 1024, 1024, 8)
+    x = (x.astype(np.float32) * 900.0).clip(-65504, 65504).astype(np.float16)
+    theta = theta * np.float32(900.0)
+    check_fused(q, s, z, x, theta, 8)

@@ -2,6 +2,8 @@
 
 Bit-exact: planes, unpack(planes), b, the per-plane lists and counts.
 Within |y - y_ref| <= 1e-3 * sum_i |w_hat_io||x_i| + 1e-6: y.
+Every case runs on both paths: grinqh_assign + grinqh_gemv ("two") and the
+fused single-kernel grinqh_decode_gemv ("fused").
 """
 import numpy as np
 import pytest
@@ -16,6 +18,7 @@ from input_adaptive_bit_b200 import (ERR_DEVICE, GrinqhError, grinqh_check_devic
 from input_adaptive_bit_b200.layer import Dense4Linear, GrinqhLinear
 
 pytestmark = pytest.mark.gpu
+PATHS = ["two", "fused"]
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -59,48 +62,55 @@ def random_case(seed, d_in, d_out, b_max, x_kind="normal", theta_kind="quantile"
 
 # ---- the parity workload ----------------------------------------------------------
 
-def test_config0_parity_everything():
+@pytest.mark.parametrize("path", PATHS)
+def test_config0_parity_everything(path):
     case = synth.make_case(synth.config0()[0])
-    lin, out = full_case_check(case)
+    lin, out = full_case_check(case, path=path)
     assert abs(oracle.effective_bits(out["b"]) - 3.3) < 0.05
 
 
 @pytest.mark.parametrize("b_max", [2, 4, 6, 8])
 @pytest.mark.parametrize("shape", [(128, 16), (256, 48), (384, 592), (1152, 1040), (2048, 512)])
-def test_random_shapes(b_max, shape):
+@pytest.mark.parametrize("path", PATHS)
+def test_random_shapes(b_max, shape, path):
     d_in, d_out = shape
-    full_case_check(random_case(1000 * b_max + d_in + d_out, d_in, d_out, b_max))
+    full_case_check(random_case(1000 * b_max + d_in + d_out, d_in, d_out, b_max), path=path)
 
 
 @pytest.mark.parametrize("theta_kind", ["ties", "zero", "inf", "decreasing", "nan"])
 @pytest.mark.parametrize("x_kind", ["normal", "special"])
-def test_adversarial_thresholds_and_inputs(theta_kind, x_kind):
-    full_case_check(random_case(7, 1280, 1040, 8, x_kind=x_kind, theta_kind=theta_kind))
+@pytest.mark.parametrize("path", PATHS)
+def test_adversarial_thresholds_and_inputs(theta_kind, x_kind, path):
+    full_case_check(random_case(7, 1280, 1040, 8, x_kind=x_kind, theta_kind=theta_kind), path=path)
 
 
-def test_random_shape_sweep():
+@pytest.mark.parametrize("path", PATHS)
+def test_random_shape_sweep(path):
     g = np.random.default_rng(123)
     for k in range(12):
         d_in = 128 * int(g.integers(1, 9))
         d_out = 16 * int(g.integers(1, 65))
         b_max = int(g.choice([2, 4, 6, 8]))
-        full_case_check(random_case(5000 + k, d_in, d_out, b_max))
+        full_case_check(random_case(5000 + k, d_in, d_out, b_max), path=path)
 
 
-def test_all_rows_skipped_gives_exact_zeros():
+@pytest.mark.parametrize("path", PATHS)
+def test_all_rows_skipped_gives_exact_zeros(path):
     case = random_case(9, 1024, 2048, 8, theta_kind="inf")
-    lin, out = run_layer(case.q, case.s, case.z, case.x, case.theta, 8)
+    lin, out = run_layer(case.q, case.s, case.z, case.x, case.theta, 8, path=path)
     assert (out["b"] == 0).all() and (out["counts"] == 0).all()
     assert (out["y"] == 0.0).all() and not np.signbit(out["y"]).any()
 
 
-def test_explicit_phi_table():
+@pytest.mark.parametrize("path", PATHS)
+def test_explicit_phi_table(path):
     case = random_case(10, 1024, 1024, 8)
     phi = np.array([0.0, 31.5, 7.5, 1.5, 0.0], np.float32)
-    full_case_check(case, phi=phi)
+    full_case_check(case, phi=phi, path=path)
 
 
-def test_one_hot_rows_recover_the_reconstructed_row():
+@pytest.mark.parametrize("path", PATHS)
+def test_one_hot_rows_recover_the_reconstructed_row(path):
     # x = e_i, b_i = 8/6/4/2: y must be the reconstructed row s(Q+phi)+z up to a
     # few fp32 roundings of its terms
     case = random_case(11, 512, 1024, 8)
@@ -110,7 +120,7 @@ def test_one_hot_rows_recover_the_reconstructed_row():
         x = np.zeros(512, np.float16)
         x[i] = 1.0
         theta = np.array([0.5] * lvl + [np.inf] * (4 - lvl), np.float32)
-        _, out = run_layer(None, None, None, x, theta, 8, lin=lin)
+        _, out = run_layer(None, None, None, x, theta, 8, lin=lin, path=path)
         b = 2 * lvl
         d = 8 - b
         Q = ((case.q[i].astype(np.int64) >> d) << d).astype(np.float64)
@@ -121,39 +131,43 @@ def test_one_hot_rows_recover_the_reconstructed_row():
         assert oracle.within_tolerance(out["y"], row, np.abs(row), REL, ABS).all()
 
 
-def test_zeroing_skipped_inputs_changes_nothing():
+@pytest.mark.parametrize("path", PATHS)
+def test_zeroing_skipped_inputs_changes_nothing(path):
     case = random_case(12, 1024, 1536, 8)
-    lin, out1 = run_layer(case.q, case.s, case.z, case.x, case.theta, 8)
+    lin, out1 = run_layer(case.q, case.s, case.z, case.x, case.theta, 8, path=path)
     x2 = case.x.copy()
     b = out1["b"]
     # |x| below theta_1 keeps b = 0 when scaled towards zero
     x2[b == 0] = (x2[b == 0].astype(np.float32) * 0.25).astype(np.float16)
-    _, out2 = run_layer(None, None, None, x2, case.theta, 8, lin=lin)
+    _, out2 = run_layer(None, None, None, x2, case.theta, 8, lin=lin, path=path)
     assert np.array_equal(out2["b"], b)
     assert np.array_equal(out1["y"], out2["y"])
 
 
-def test_deterministic_across_calls():
+@pytest.mark.parametrize("path", PATHS)
+def test_deterministic_across_calls(path):
     case = random_case(13, 4096, 4096, 8)
-    lin, out1 = run_layer(case.q, case.s, case.z, case.x, case.theta, 8)
+    lin, out1 = run_layer(case.q, case.s, case.z, case.x, case.theta, 8, path=path)
     for _ in range(3):
-        _, out2 = run_layer(None, None, None, case.x, case.theta, 8, lin=lin)
+        _, out2 = run_layer(None, None, None, case.x, case.theta, 8, lin=lin, path=path)
         assert np.array_equal(out1["y"], out2["y"])
         assert np.array_equal(out1["grp_sums"], out2["grp_sums"])
 
 
-def test_scaling_x_and_theta_by_power_of_two():
+@pytest.mark.parametrize("path", PATHS)
+def test_scaling_x_and_theta_by_power_of_two(path):
     case = random_case(14, 1024, 1024, 8)
     x = case.x.astype(np.float32)
     x = (np.sign(x) * np.maximum(np.abs(x), 0.01)).astype(np.float16)
-    lin, out1 = run_layer(case.q, case.s, case.z, x, case.theta, 8)
+    lin, out1 = run_layer(case.q, case.s, case.z, x, case.theta, 8, path=path)
     xs = (x.astype(np.float32) * 4).astype(np.float16)
-    _, out2 = run_layer(None, None, None, xs, case.theta * np.float32(4), 8, lin=lin)
+    _, out2 = run_layer(None, None, None, xs, case.theta * np.float32(4), 8, lin=lin, path=path)
     assert np.array_equal(out1["b"], out2["b"])
     assert np.array_equal(out1["y"] * 4, out2["y"])
 
 
-def test_workspace_shared_by_layers_of_different_shapes():
+@pytest.mark.parametrize("path", PATHS)
+def test_workspace_shared_by_layers_of_different_shapes(path):
     big = random_case(15, 2048, 4096, 8)
     small = random_case(16, 512, 1024, 6)
     lin_b = GrinqhLinear(big.q, big.s, big.z, 8)
@@ -161,7 +175,7 @@ def test_workspace_shared_by_layers_of_different_shapes():
     lin_s.ws = lin_b.ws  # one workspace sized for the largest layer
     lin_s.ws_bytes = lin_b.ws_bytes
     for case, lin in [(small, lin_s), (big, lin_b), (small, lin_s)]:
-        _, out = run_layer(None, None, None, case.x, case.theta, lin.b_max, lin=lin)
+        _, out = run_layer(None, None, None, case.x, case.theta, lin.b_max, lin=lin, path=path)
         b_ref = check_assign(out, case.x, case.theta, lin.b_max)
         check_y(out, oracle.pack(case.q, lin.b_max), case.s, case.z, case.x, b_ref, lin.b_max)
     grinqh_check_device_error(lin_b.ws)
@@ -203,40 +217,44 @@ def test_dense4_comparator_parity():
 
 @pytest.mark.slow
 @pytest.mark.parametrize("idx", range(12))
-def test_qwen3_8b_projections(idx):
+@pytest.mark.parametrize("path", PATHS)
+def test_qwen3_8b_projections(idx, path):
     lin = synth.config1()[idx]
     case = synth.make_case(lin)
-    _, out = full_case_check(case, sample_outputs=256, sample_rows=64)
+    _, out = full_case_check(case, sample_outputs=256, sample_rows=64, path=path)
     assert abs(oracle.effective_bits(out["b"]) - lin.target_bits) < 0.1
 
 
 @pytest.mark.slow
 @pytest.mark.parametrize("idx", range(7))
-def test_uniform_sweep_llama_up_proj(idx):
+@pytest.mark.parametrize("path", PATHS)
+def test_uniform_sweep_llama_up_proj(idx, path):
     lin = synth.config2()[idx]
     case = synth.make_case(lin)
-    _, out = full_case_check(case, sample_outputs=256, sample_rows=64)
+    _, out = full_case_check(case, sample_outputs=256, sample_rows=64, path=path)
     if lin.uniform_b is not None:
         assert (out["b"] == lin.uniform_b).all()
 
 
 @pytest.mark.slow
 @pytest.mark.parametrize("idx", [0, 1, 3, 5])
-def test_70b_shapes_redrawn_inputs(idx):
+@pytest.mark.parametrize("path", PATHS)
+def test_70b_shapes_redrawn_inputs(idx, path):
     spec = synth.config3()[idx]
     case = synth.make_case(spec)
-    lin, _ = full_case_check(case, sample_outputs=128, sample_rows=32)
+    lin, _ = full_case_check(case, sample_outputs=128, sample_rows=32, path=path)
     planes_ref = oracle.pack(case.q, spec.b_max)
     for call in (1, 2):  # a fresh x per call changes the active rows
         x = synth.make_x(spec, call)
-        _, out = run_layer(None, None, None, x, case.theta, spec.b_max, lin=lin)
+        _, out = run_layer(None, None, None, x, case.theta, spec.b_max, lin=lin, path=path)
         b_ref = check_assign(out, x, case.theta, spec.b_max)
         outs = np.random.default_rng(call).integers(0, spec.d_out, 64).astype(np.int32)
         check_y(out, planes_ref, case.s, case.z, x, b_ref, spec.b_max, outs=outs)
 
 
 @pytest.mark.slow
-def test_llama3_8b_layer_of_the_decode_step():
+@pytest.mark.parametrize("path", PATHS)
+def test_llama3_8b_layer_of_the_decode_step(path):
     for spec in synth.config4(n_layers=1):
         case = synth.make_case(spec)
-        full_case_check(case, sample_outputs=128, sample_rows=32)
+        full_case_check(case, sample_outputs=128, sample_rows=32, path=path)
