@@ -53,10 +53,11 @@ constexpr int kStage = 64;            // units per ring stage (4 k-steps, 2 per 
 constexpr int kRing = 8;              // ring stages
 constexpr int kRingEarly = 6;         // stages issued before the x cache (on the last slots) is freed
 constexpr int kRound = 1024;          // units per round
-constexpr int kSlots = 8;             // groups per round (the MMA n dimension)
+constexpr int kSlots = 8;             // groups per window (the MMA n dimension)
 constexpr int kMaxG = kDecodeMaxDin / kGroup;
-constexpr int kXCache = 16384;        // rows of x held in shared memory (larger d_in: in chunks)
-constexpr int kGT = 16;               // front-end threads per group (8 rows each)
+constexpr int kXCache = 16384;        // rows of x held in shared memory
+constexpr int kGT = 16;               // threads per group: one 8-row chunk each
+constexpr int kOutCtas = 4;           // CTAs that write the optional outputs
 
 // shared memory map (bytes)
 constexpr size_t kStageBytes = (size_t)kStage * kRow * 4;
@@ -68,28 +69,30 @@ constexpr size_t kSmUx = kSmRegion + kRound * 4;                            // u
 constexpr size_t kSmBfrag = kSmUx + kRound * 4;                             // uint2 [kRound / kK][32]
 constexpr size_t kSmS = kSmBfrag + (size_t)(kRound / kK) * 32 * 8;          // fp16 [kSlots][kTile]
 constexpr size_t kSmZ = kSmS + (size_t)kSlots * kTile * 2;                  // fp16 [kSlots][kTile]
-constexpr size_t kSmCnt = kSmZ + (size_t)kSlots * kTile * 2;                // u32 [kMaxG]: plane counts, bytes
-constexpr size_t kSmLoff = kSmCnt + (size_t)kMaxG * 4;                      // int4 [kMaxG]: list offsets
-constexpr size_t kSmGoff = kSmLoff + (size_t)kMaxG * 16;                    // i32 [kMaxG + 4]: unit offsets
-constexpr size_t kSmSlot = kSmGoff + (size_t)(kMaxG + 4) * 4;               // SlotInfo [kSlots]
-constexpr size_t kSmWsum = kSmSlot + kSlots * 16;                           // int4 [kWarps]
-constexpr size_t kSmRed = kSmWsum + kWarps * 16;                            // fp32 [kTile]: odd-k warps
+constexpr size_t kSmSlot = kSmZ + (size_t)kSlots * kTile * 2;               // SlotInfo [kSlots]
+constexpr size_t kSmTot = kSmSlot + kSlots * 16;                            // i32 [kSlots][4]: window units
+constexpr size_t kSmRed = kSmTot + kSlots * 16;                             // fp32 [kTile]: odd-k warps
 constexpr size_t kSmBytes = kSmRed + (size_t)kTile * 4;
+// the output CTAs keep their counts and scans where the GEMV CTAs have the ring
+constexpr size_t kSmCnt = kSmRing;                                          // u32 [kMaxG]: plane counts, bytes
+constexpr size_t kSmLoff = kSmCnt + (size_t)kMaxG * 4;                      // int4 [kMaxG]: list offsets
+constexpr size_t kSmWsum = kSmLoff + (size_t)kMaxG * 16;                    // int4 [kWarps]
 static_assert(kSmBytes <= 227 * 1024, "shared memory");
 static_assert((size_t)kXCache * 2 <= (size_t)(kRing - kRingEarly) * kStageBytes, "x cache fits");
+static_assert(kSmWsum + kWarps * 16 <= kSmX, "output-CTA arrays below the x cache");
 static_assert(kSmRing % 16 == 0 && kSmX % 16 == 0 && kSmS % 16 == 0 && kSmZ % 16 == 0 &&
-                  kSmBfrag % 16 == 0 && kSmCnt % 16 == 0 && kSmLoff % 16 == 0 && kSmSlot % 16 == 0 &&
+                  kSmBfrag % 16 == 0 && kSmLoff % 16 == 0 && kSmSlot % 16 == 0 &&
                   kSmWsum % 16 == 0 && kSmRed % 16 == 0,
               "16-byte aligned regions");
 static_assert(kStage * 16 == 2 * kThreads, "two 16-byte copies per thread and stage");
 static_assert(kStage == 4 * kK && kWarps == 2 * kBlocks, "two k-steps per warp and stage");
-static_assert(kSlots * kGT <= kThreads && kMaxG == kThreads, "thread mappings");
+static_assert(kMaxG == kThreads, "one group per thread in the output CTAs' scan");
 
 struct SlotInfo {
   int c;       // the group's B-column scale exponent: B holds x 4^(P-1-p) 2^-c
-  float X;     // sum of x over the group's active rows (added if `first`)
-  float Phi;   // sum of x phi_{b/2} over the group's active rows
-  int first;   // the group's first unit lies in this round: add s Phi + z X here
+  float X;     // sum of x over the active rows of the group in this CTA's row slice
+  float Phi;   // sum of x phi_{b/2} over the same rows
+  int pad;
 };
 
 struct DecodeArgs {
@@ -140,8 +143,6 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-__device__ __forceinline__ float h2f(uint16_t h) { return __half2float(__ushort_as_half(h)); }
-
 // 2^e as a float, for |e| well inside the normal range.
 __device__ __forceinline__ float exp2i(int e) { return __int_as_float((127 + e) << 23); }
 
@@ -152,98 +153,54 @@ __host__ __device__ constexpr int field_pos(int t) {
   return (t & 7) <= 4 ? 2 * (t & 7) : 2 * (t & 7) - 6;
 }
 
-template <bool ALIGNED>
-__global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
-  extern __shared__ __align__(128) unsigned char smem[];
-  uint32_t *ring = reinterpret_cast<uint32_t *>(smem + kSmRing);
+// The optional outputs (b, lists, counts, group sums): written by CTAs that
+// take no part in the GEMV, so they cost the GEMV nothing but those CTAs' SMs.
+// Every output CTA counts the units of every group per plane and scans them
+// (the list offsets); then CTA k of K writes the groups g = k mod K.
+__device__ __forceinline__ void write_outputs(const DecodeArgs &a, unsigned char *smem, int k,
+                                              int K, const __half2 (&t2)[4],
+                                              const float (&phi)[5]) {
   uint16_t *xc = reinterpret_cast<uint16_t *>(smem + kSmX);
-  int32_t *s_region = reinterpret_cast<int32_t *>(smem + kSmRegion);
-  uint32_t *s_ux = reinterpret_cast<uint32_t *>(smem + kSmUx);
-  uint2 *s_bfrag = reinterpret_cast<uint2 *>(smem + kSmBfrag);
-  uint16_t *s_st = reinterpret_cast<uint16_t *>(smem + kSmS);
-  uint16_t *z_st = reinterpret_cast<uint16_t *>(smem + kSmZ);
   uint32_t *s_cnt = reinterpret_cast<uint32_t *>(smem + kSmCnt);
   int4 *s_loff = reinterpret_cast<int4 *>(smem + kSmLoff);
-  int *s_goff = reinterpret_cast<int *>(smem + kSmGoff);
-  SlotInfo *s_slot = reinterpret_cast<SlotInfo *>(smem + kSmSlot);
   int4 *s_wsum = reinterpret_cast<int4 *>(smem + kSmWsum);
-  float *s_red = reinterpret_cast<float *>(smem + kSmRed);
-  __shared__ int s_last;
-
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int fg = lane >> 2, tq = lane & 3;  // MMA fragment row group and column pair
-  const int ob = warp & (kBlocks - 1);      // the warp's 128-output block of the tile
-  const int kp = warp / kBlocks;            // ... and its k-step parity
-  const int gsub = tid & (kGT - 1);         // front end: lane of a 16-thread group team
-  const int C = gridDim.x, c = blockIdx.x;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, gsub = tid & (kGT - 1);
   const int P = a.P, G = a.G;
-
-  // x, theta and the weights may be written by the kernel launched just before
-  asm volatile("griddepcontrol.wait;\n" ::: "memory");
-
-  __half2 t2[4];
-  make_thresholds(a.theta, P, t2);
-  float phi[5];
-#pragma unroll
-  for (int k = 0; k <= 4; ++k) {
-    const float def = (2 * k < a.b_max) ? exp2i(a.b_max - 2 * k - 1) : 0.0f;
-    phi[k] = (k <= P) ? (a.phi ? a.phi[k] : def) : 0.0f;
-  }
-
-  // rows 128 g + 8 gsub .. + 7 of x: from the shared cache while it holds them
   int xc_base = 0;
-  bool xc_valid = true;
   auto load8 = [&](int g) -> uint4 {
     const int row = g * kGroup + 8 * gsub;
-    if (xc_valid && row >= xc_base && row < xc_base + kXCache)
+    if (row >= xc_base && row < xc_base + kXCache)
       return *reinterpret_cast<const uint4 *>(xc + (row - xc_base));
     return __ldg(reinterpret_cast<const uint4 *>(a.x + row));
   };
-
-  // ---- units per (group, plane) ----------------------------------------------------
-  // x goes to shared memory in one cp.async wave per chunk of kXCache rows; 16
-  // threads count a group (8 rows each), the four plane counts (each <= 128)
-  // packed into the bytes of one word; two groups per team and pass.
+  // units per (group, plane), x in chunks of kXCache rows
   for (int base = 0; base < a.d_in; base += kXCache) {
     const int rows = min(kXCache, a.d_in - base);
-    if (base > 0) __syncthreads();  // the previous chunk is counted
+    if (base > 0) __syncthreads();
     for (int q = tid; q < rows / 8; q += kThreads) cp_async16(xc + 8 * q, a.x + base + 8 * q, 16);
     cp_async_commit();
     cp_async_wait<0>();
     __syncthreads();
     xc_base = base;
     const int g_lo = base / kGroup, g_hi = (base + rows) / kGroup;
-    for (int g0 = g_lo; g0 < g_hi; g0 += 2 * (kThreads / kGT)) {
-      const int ga = g0 + (tid >> 4), gb = ga + kThreads / kGT;
-      uint32_t pa = 0, pb = 0;
-      uint32_t ma[4], mb[4];
-      plane_masks8(ga < g_hi ? load8(ga) : make_uint4(0, 0, 0, 0), t2, P, ma);
-      plane_masks8(gb < g_hi ? load8(gb) : make_uint4(0, 0, 0, 0), t2, P, mb);
+    for (int g0 = g_lo; g0 < g_hi; g0 += kThreads / kGT) {
+      const int g = g0 + (tid >> 4);
+      uint32_t mk[4] = {0u, 0u, 0u, 0u};
+      if (g < g_hi) plane_masks8(load8(g), t2, P, mk);
+      uint32_t packed = 0;
 #pragma unroll
-      for (int p = 0; p < 4; ++p) {
-        pa += (uint32_t)__popc(ma[p]) << (8 * p);
-        pb += (uint32_t)__popc(mb[p]) << (8 * p);
-      }
+      for (int p = 0; p < 4; ++p) packed += (uint32_t)__popc(mk[p]) << (8 * p);
 #pragma unroll
-      for (int off = 8; off > 0; off >>= 1) {
-        pa += __shfl_xor_sync(0xffffffffu, pa, off);
-        pb += __shfl_xor_sync(0xffffffffu, pb, off);
-      }
-      if (gsub == 0 && ga < g_hi) s_cnt[ga] = pa;
-      if (gsub == 0 && gb < g_hi) s_cnt[gb] = pb;
+      for (int off = 8; off > 0; off >>= 1) packed += __shfl_xor_sync(0xffffffffu, packed, off);
+      if (gsub == 0 && g < g_hi) s_cnt[g] = packed;
     }
   }
-  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
   __syncthreads();
-
-  // ---- exclusive scans over groups: per-plane list offsets and unit offsets ----
+  // exclusive scans over groups: per-plane list offsets
   {
     const int g0 = tid;  // kMaxG = kThreads
-    auto unpack = [](uint32_t v) {
-      return make_int4(v & 255u, (v >> 8) & 255u, (v >> 16) & 255u, v >> 24);
-    };
-    const int4 z4 = make_int4(0, 0, 0, 0);
-    const int4 v0 = g0 < G ? unpack(s_cnt[g0]) : z4;
+    const uint32_t v = g0 < G ? s_cnt[g0] : 0u;
+    const int4 v0 = make_int4(v & 255u, (v >> 8) & 255u, (v >> 16) & 255u, v >> 24);
     int4 inc = v0;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
@@ -256,147 +213,190 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
     }
     if (lane == 31) s_wsum[warp] = inc;
     __syncthreads();
-    int4 pre = z4, tot = z4;
+    int4 pre = make_int4(0, 0, 0, 0), tot = pre;
 #pragma unroll
     for (int w = 0; w < kWarps; ++w) {
       const int4 t = s_wsum[w];
       if (w < warp) pre = make_int4(pre.x + t.x, pre.y + t.y, pre.z + t.z, pre.w + t.w);
       tot = make_int4(tot.x + t.x, tot.y + t.y, tot.z + t.z, tot.w + t.w);
     }
-    const int4 ex0 = make_int4(pre.x + inc.x - v0.x, pre.y + inc.y - v0.y,
-                               pre.z + inc.z - v0.z, pre.w + inc.w - v0.w);
-    if (g0 < G) {
-      s_loff[g0] = ex0;
-      s_goff[g0] = ex0.x + ex0.y + ex0.z + ex0.w;
-    }
-    if (tid == 0) {
-      s_goff[G] = tot.x + tot.y + tot.z + tot.w;
-      if (c == 0 && a.counts) {
-        if (P > 0) a.counts[0] = tot.x;
-        if (P > 1) a.counts[1] = tot.y;
-        if (P > 2) a.counts[2] = tot.z;
-        if (P > 3) a.counts[3] = tot.w;
-      }
+    if (g0 < G)
+      s_loff[g0] = make_int4(pre.x + inc.x - v0.x, pre.y + inc.y - v0.y, pre.z + inc.z - v0.z,
+                             pre.w + inc.w - v0.w);
+    if (tid == 0 && k == 0 && a.counts) {
+      if (P > 0) a.counts[0] = tot.x;
+      if (P > 1) a.counts[1] = tot.y;
+      if (P > 2) a.counts[2] = tot.z;
+      if (P > 3) a.counts[3] = tot.w;
     }
     __syncthreads();
   }
-  const int U = s_goff[G];
-
-  // ---- optional outputs (b, lists, group sums) -------------------------------------
-  // team t (16 threads) of CTA c writes group c + C t, so the work is spread one
-  // group per CTA first; run where it hides under memory latency (after a
-  // round's first copies are issued), by CTAs without GEMV work first thing
-  bool outputs_pending = a.b || a.lists || a.grp_sums;
-  auto write_outputs = [&]() {
-    outputs_pending = false;
-    // the same number of passes for every thread (the shuffles span whole warps)
-    for (int g0 = 0; g0 < G; g0 += C * (kThreads / kGT)) {
-      const int g = g0 + c + C * (tid >> 4);
-      const bool act = g < G;
-      const uint4 xw = act ? load8(g) : make_uint4(0, 0, 0, 0);
-      uint32_t mk[4];
-      plane_masks8(xw, t2, P, mk);
-      const int row0 = g * kGroup + 8 * gsub;
-      if (a.grp_sums) {
-        float X, Phi;
-        group_sums8(xw, mk, phi, X, Phi);
-        if (act && gsub == 0) {
-          a.grp_sums[g] = X;
-          a.grp_sums[G + g] = Phi;
-        }
+  // team t (16 threads) of output CTA k writes group k + K (t + 32 pass)
+  for (int g0 = 0; g0 + k < G; g0 += K * (kThreads / kGT)) {
+    const int g = g0 + k + K * (tid >> 4);
+    const bool act = g < G;
+    const uint4 xw = act ? load8(g) : make_uint4(0, 0, 0, 0);
+    uint32_t mk[4] = {0u, 0u, 0u, 0u};
+    if (act) plane_masks8(xw, t2, P, mk);
+    const int row0 = g * kGroup + 8 * gsub;
+    if (a.grp_sums) {
+      float X, Phi;
+      group_sums8(xw, mk, phi, X, Phi);
+      if (act && gsub == 0) {
+        a.grp_sums[g] = X;
+        a.grp_sums[G + g] = Phi;
       }
-      if (a.b && act) {
+    }
+    if (a.b && act) {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) a.b[row0 + e] = (uint8_t)(2 * row_level(mk, e));
+      for (int e = 0; e < 8; ++e) a.b[row0 + e] = (uint8_t)(2 * row_level(mk, e));
+    }
+    if (a.lists) {
+      uint32_t cnt = 0;
+#pragma unroll
+      for (int p = 0; p < 4; ++p) cnt += (uint32_t)__popc(mk[p]) << (8 * p);
+      uint32_t inc = cnt;
+#pragma unroll
+      for (int off = 1; off < kGT; off <<= 1) {
+        const uint32_t t = __shfl_up_sync(0xffffffffu, inc, off, kGT);
+        if (gsub >= off) inc += t;
       }
-      if (a.lists) {
-        uint32_t cnt = 0;
+      const uint32_t pre = inc - cnt;
+      if (act) {
+        const int4 lo = s_loff[g];
+        const int lofs[4] = {lo.x, lo.y, lo.z, lo.w};
 #pragma unroll
-        for (int p = 0; p < 4; ++p) cnt += (uint32_t)__popc(mk[p]) << (8 * p);
-        uint32_t inc = cnt;
+        for (int p = 0; p < 4; ++p) {
+          if (p >= P) break;
+          int pos = lofs[p] + (int)((pre >> (8 * p)) & 255u);
+          int32_t *lp = a.lists + (size_t)p * a.d_in;
 #pragma unroll
-        for (int off = 1; off < kGT; off <<= 1) {
-          const uint32_t t = __shfl_up_sync(0xffffffffu, inc, off, kGT);
-          if (gsub >= off) inc += t;
-        }
-        const uint32_t pre = inc - cnt;
-        if (act) {
-          const int4 lo = s_loff[g];
-          const int lofs[4] = {lo.x, lo.y, lo.z, lo.w};
-#pragma unroll
-          for (int p = 0; p < 4; ++p) {
-            if (p >= P) break;
-            int pos = lofs[p] + (int)((pre >> (8 * p)) & 255u);
-            int32_t *lp = a.lists + (size_t)p * a.d_in;
-#pragma unroll
-            for (int e = 0; e < 8; ++e)
-              if ((mk[p] >> e) & 1u) lp[pos++] = row0 + e;
-          }
+          for (int e = 0; e < 8; ++e)
+            if ((mk[p] >> e) & 1u) lp[pos++] = row0 + e;
         }
       }
     }
+  }
+}
+
+template <bool ALIGNED>
+__global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  uint32_t *ring = reinterpret_cast<uint32_t *>(smem + kSmRing);
+  uint16_t *xc = reinterpret_cast<uint16_t *>(smem + kSmX);
+  int32_t *s_region = reinterpret_cast<int32_t *>(smem + kSmRegion);
+  uint32_t *s_ux = reinterpret_cast<uint32_t *>(smem + kSmUx);
+  uint2 *s_bfrag = reinterpret_cast<uint2 *>(smem + kSmBfrag);
+  uint16_t *s_st = reinterpret_cast<uint16_t *>(smem + kSmS);
+  uint16_t *z_st = reinterpret_cast<uint16_t *>(smem + kSmZ);
+  SlotInfo *s_slot = reinterpret_cast<SlotInfo *>(smem + kSmSlot);
+  int *s_tot = reinterpret_cast<int *>(smem + kSmTot);
+  float *s_red = reinterpret_cast<float *>(smem + kSmRed);
+  __shared__ int s_last;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int fg = lane >> 2, tq = lane & 3;  // MMA fragment row group and column pair
+  const int ob = warp & (kBlocks - 1);      // the warp's 128-output block of the tile
+  const int kp = warp / kBlocks;            // ... and its k-step parity
+  const int gsub = tid & (kGT - 1);
+  const int C = gridDim.x, c = blockIdx.x;
+  const int P = a.P;
+
+  // x, theta and the weights may be written by the kernel launched just before
+  asm volatile("griddepcontrol.wait;\n" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+
+  // thresholds and phi (loaded where their latency hides behind copies in flight)
+  __half2 t2[4];
+  float phi[5];
+  auto load_thresholds = [&]() {
+    make_thresholds(a.theta, P, t2);
+#pragma unroll
+    for (int k = 0; k <= 4; ++k) {
+      const float def = (2 * k < a.b_max) ? exp2i(a.b_max - 2 * k - 1) : 0.0f;
+      phi[k] = (k <= P) ? (a.phi ? a.phi[k] : def) : 0.0f;
+    }
   };
 
-  if (U == 0) {  // no active row: y = 0 exactly
-    if (outputs_pending) write_outputs();
-    for (int o = c * kThreads + tid; o < a.d_out; o += C * kThreads) a.y[o] = 0.0f;
+  // the last CTAs write the optional outputs, the others run the GEMV; they are
+  // set aside whether or not outputs are asked for, so y does not depend on it
+  const int n_out = C > 2 * kOutCtas ? kOutCtas : 1;
+  const int C_g = C - n_out;
+  if (c >= C_g) {
+    if (a.b || a.lists || a.counts || a.grp_sums) {
+      load_thresholds();
+      write_outputs(a, smem, c - C_g, n_out, t2, phi);
+    }
     return;
   }
+  bool thresholds_loaded = false;
 
-  // m CTAs per tile (m <= U, so no range is empty); more tiles than CTAs: whole tiles in turn
-  const int m = a.tiles >= C ? 1 : min(C / a.tiles, U);
-  const int C_eff = a.tiles >= C ? C : a.tiles * m;
-  if (c >= C_eff) {
-    if (outputs_pending) write_outputs();
-    return;
-  }
+  // tiles x row slices: m CTAs per tile, CTA `part` takes the 8-row chunks
+  // [R8 part / m, R8 (part + 1) / m); more tiles than CTAs: whole tiles in turn
+  const bool many = a.tiles >= C_g;
+  const int m = many ? 1 : C_g / a.tiles;
+  const int C_eff = many ? C_g : a.tiles * m;
+  if (c >= C_eff) return;
+  const int R8 = a.d_in / 8;
+  const int part = many ? 0 : c % m;
+  const int q_lo = R8 * part / m, q_hi = R8 * (part + 1) / m;  // R8 <= 2^13, part < 2^8
+  const int row_lo = 8 * q_lo, row_hi = 8 * q_hi;
 
-  for (int tile = c / m; tile < a.tiles; tile += C_eff / m) {
-    const int part = c % m;
-    // U <= 2^18 and part < 256: the products fit 32 bits
-    const int u0 = part * U / m, u1 = (part + 1) * U / m;
+  // the slice of x to shared memory when it fits (else it is read from global memory)
+  bool xc_valid = row_hi - row_lo <= kXCache;
+  if (xc_valid)
+    for (int q = tid; q < q_hi - q_lo; q += kThreads) cp_async16(xc + 8 * q, a.x + row_lo + 8 * q, 16);
+  cp_async_commit();
+
+  for (int tile = many ? c : c / m; tile < a.tiles; tile += many ? C_g : a.tiles) {
     const int wbase = tile * kTileW;  // first word of the tile in a plane region
-
     float yacc[16];
 #pragma unroll
     for (int t = 0; t < 16; ++t) yacc[t] = 0.0f;
 
-    for (int r0 = u0, r1; r0 < u1; r0 = r1) {
-      // the round: units [r0, r1) of at most kRound units and kSlots groups
-      int lo = 0, hi = G;  // largest g with goff[g] <= r0 (a non-empty group holds r0)
-      while (hi - lo > 1) {
-        const int mid = (lo + hi) >> 1;
-        if (s_goff[mid] <= r0) lo = mid; else hi = mid;
-      }
-      const int g_first = lo, g_end = min(g_first + kSlots, G), ng = g_end - g_first;
-      r1 = min(u1, min(r0 + kRound, s_goff[g_end]));
-      const int n = r1 - r0, n_pad = (n + kK - 1) & ~(kK - 1);
-      const int n_steps = n_pad / kK, n_stages = (n_pad + kStage - 1) / kStage;
+    // windows of kSlots groups over the slice
+    for (int g_w = row_lo / kGroup; g_w * kGroup < row_hi; g_w += kSlots) {
+      const int ng = min(kSlots, (row_hi + kGroup - 1) / kGroup - g_w);
+      __syncthreads();  // the previous window no longer reads the staged data
 
-      __syncthreads();  // the previous round no longer reads the staged data
-
-      // stage s and z rows of the round's groups for this tile (rows past d_out: zero)
+      // stage s and z rows of the window's groups for this tile (past d_out: zero)
 #pragma unroll
       for (int i = 0; i < 2 * kSlots * (kTile / 8) / kThreads; ++i) {
         const int q = tid + i * kThreads;  // [which][slot][chunk of 8 halves]
         const int which = q / (kSlots * (kTile / 8)), gi = (q / (kTile / 8)) % kSlots;
         const int ci = q % (kTile / 8), o = tile * kTile + ci * 8;
         if (gi < ng) {
-          const uint16_t *src = (which ? a.z : a.s) + (size_t)(g_first + gi) * a.d_out + o;
+          const uint16_t *src = (which ? a.z : a.s) + (size_t)(g_w + gi) * a.d_out + o;
           uint16_t *dst = (which ? z_st : s_st) + gi * kTile + ci * 8;
           cp_async16(dst, o < a.d_out ? (const void *)src : (const void *)a.s, o < a.d_out ? 16 : 0);
         }
       }
       cp_async_commit();
+      if (!thresholds_loaded) {
+        load_thresholds();
+        thresholds_loaded = true;
+      }
+      cp_async_wait<1>();  // the x slice (committed before) has landed
+      __syncthreads();
 
-      // compaction of the round's groups: a 16-thread team per group slot
-      if (tid < kSlots * kGT) {
-        const int gi = tid >> 4, g = g_first + gi;
-        const bool act = gi < ng && s_goff[g] < r1 && s_goff[g + 1] > r0;
-        const uint4 xw = act ? load8(g) : make_uint4(0, 0, 0, 0);
-        uint32_t mk[4];
+      // compaction: a 16-thread team per (group slot, plane); thread gsub of team
+      // (slot, pl) takes chunk 16 (g_w + slot) + gsub of the window and that
+      // chunk's units of plane pl.  Units are placed slot by slot, then plane by
+      // plane, then chunk by chunk, then row by row (the order within a round is free)
+      static_assert(kSlots * 4 * kGT == kThreads, "one team per slot and plane");
+      const int slot = tid >> 6, pl = (tid >> 4) & 3;
+      const int qc = kGT * (g_w + slot) + gsub;  // the thread's chunk
+      const bool act = qc >= q_lo && qc < q_hi;
+      uint4 xw = make_uint4(0, 0, 0, 0);
+      uint32_t mk[4] = {0u, 0u, 0u, 0u};
+      if (act) {
+        xw = xc_valid ? *reinterpret_cast<const uint4 *>(xc + 8 * (qc - q_lo))
+                      : __ldg(reinterpret_cast<const uint4 *>(a.x + 8 * qc));
         plane_masks8(xw, t2, P, mk);
-        // B-column scale: the largest active |x| times 4^(P-1) stays below 2^16
+      }
+      int cg;
+      {
+        // B-column scale: the largest active |x| of the slot times 4^(P-1) stays below 2^16
         const uint32_t w[4] = {xw.x, xw.y, xw.z, xw.w};
         uint32_t amax = 0;
 #pragma unroll
@@ -404,193 +404,211 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
           if ((mk[0] >> e) & 1u) amax = max(amax, (w[e >> 1] >> (16 * (e & 1))) & 0x7fffu);
 #pragma unroll
         for (int off = 8; off > 0; off >>= 1) amax = max(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-        const int cg = (amax >= 0x7c00u) ? 0 : max(0, (int)(amax >> 10) - 15 + 2 * P - 16);
-        float X, Phi;
-        group_sums8(xw, mk, phi, X, Phi);
-        uint32_t cnt = 0;
-#pragma unroll
-        for (int p = 0; p < 4; ++p) cnt += (uint32_t)__popc(mk[p]) << (8 * p);
+        cg = (amax >= 0x7c00u) ? 0 : max(0, (int)(amax >> 10) - 15 + 2 * P - 16);
+      }
+      const uint32_t mp = pl == 0 ? mk[0] : pl == 1 ? mk[1] : pl == 2 ? mk[2] : mk[3];
+      const uint32_t cnt = (uint32_t)__popc(mp);
+      uint32_t pre;
+      {
         uint32_t inc = cnt;
 #pragma unroll
         for (int off = 1; off < kGT; off <<= 1) {
           const uint32_t t = __shfl_up_sync(0xffffffffu, inc, off, kGT);
           if (gsub >= off) inc += t;
         }
-        const uint32_t pre = inc - cnt;
-        if (act) {
-          const uint32_t gc = s_cnt[g];
-          int pbase = s_goff[g];
-          const int row0 = g * kGroup + 8 * gsub;
-#pragma unroll
-          for (int p = 0; p < 4; ++p) {
-            if (p >= P) break;
-            int u = pbase + (int)((pre >> (8 * p)) & 255u);
-            const float xscale = exp2i(2 * (P - 1 - p) - cg);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              if ((mk[p] >> e) & 1u) {
-                if (u >= r0 && u < r1) {
-                  const float xv = h2f((uint16_t)(w[e >> 1] >> (16 * (e & 1))));
-                  s_region[u - r0] = (row0 + e) * P + p;
-                  s_ux[u - r0] = (uint32_t)__half_as_ushort(__float2half_rn(xv * xscale)) |
-                                 ((uint32_t)gi << 16);
-                }
-                ++u;
-              }
-            }
-            pbase += (int)((gc >> (8 * p)) & 255u);
-          }
-        }
-        if (gsub == 0) {
-          SlotInfo si = {0, 0.0f, 0.0f, 0};
-          if (act) {
-            si.c = cg;
-            si.X = X;
-            si.Phi = Phi;
-            si.first = (s_goff[g] >= r0 && s_goff[g] < r1) ? 1 : 0;
-          }
-          s_slot[gi] = si;
-        }
+        pre = inc - cnt;
+        if (gsub == kGT - 1) s_tot[4 * slot + pl] = (int)inc;
       }
-      for (int k = n + tid; k < n_pad; k += kThreads) {  // padding units: no load, B = 0
-        s_region[k] = -1;
-        s_ux[k] = 0u;
+      if ((warp & 1) == 0) {  // the warps holding planes 0 and 1: the slot's group sums
+        float X, Phi;
+        group_sums8(xw, mk, phi, X, Phi);
+        if (pl == 0 && gsub == 0) {
+          SlotInfo si = {cg, X, Phi, 0};
+          s_slot[slot] = si;
+        }
       }
       __syncthreads();
+      int base = 0, Nw = 0;
+#pragma unroll
+      for (int j = 0; j < 4 * kSlots; ++j) {
+        const int t = s_tot[j];
+        base += (j < 4 * slot + pl) ? t : 0;
+        Nw += t;
+      }
+      base += (int)pre;  // this thread's first unit in the window
+      // x 4^(P-1-pl) 2^-c of the thread's 8 rows, rounded to fp16 (a power-of-two
+      // product: exact unless the result is subnormal, then rounded as fp16 does)
+      uint32_t xs[4] = {0u, 0u, 0u, 0u};
+      if (pl < P) {
+        const __half2 sc = __half2half2(__ushort_as_half((uint16_t)((15 + 2 * (P - 1 - pl) - cg) << 10)));
+        const uint32_t w[4] = {xw.x, xw.y, xw.z, xw.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const __half2 r = __hmul2(*reinterpret_cast<const __half2 *>(&w[j]), sc);
+          xs[j] = *reinterpret_cast<const uint32_t *>(&r);
+        }
+      }
 
-      // ring: stage st holds units 32 st .. 32 st + 31 of the round
-      auto issue = [&](int st) {
-        uint32_t *dst_stage = ring + (size_t)(st % kRing) * (kStage * kRow);
+      for (int k0 = 0; k0 < Nw; k0 += kRound) {
+        const int n = min(kRound, Nw - k0), n_pad = (n + kK - 1) & ~(kK - 1);
+        const int n_steps = n_pad / kK, n_stages = (n_pad + kStage - 1) / kStage;
+        if (k0 > 0) __syncthreads();  // the previous round no longer reads the records
+
+        // this thread's units that fall in [k0, k0 + n)
+        if (cnt > 0) {
+          const int rp = 8 * qc * P + pl;  // region of the chunk's row 0, plane pl
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int q = tid + h * kThreads, ul = q >> 4, part16 = q & 15;
-          const int k = st * kStage + ul;
-          const int region = k < n_pad ? s_region[k] : -1;
-          const int word = wbase + part16 * 4;
-          uint32_t *dst = dst_stage + ul * kRow + part16 * 4;
-          if (region >= 0) {
-            const uint32_t *src = a.planes + (size_t)region * a.W + word;
-            if (ALIGNED) {
-              if (word < a.W) cp_async16(dst, src, 16);
-            } else {
-#pragma unroll
-              for (int v = 0; v < 4; ++v)
-                if (word + v < a.W) cp_async4(dst + v, src + v);
+          for (int e = 0; e < 8; ++e) {
+            const int ue = base + __popc(mp & ((1u << e) - 1u));
+            if (((mp >> e) & 1u) && ue >= k0 && ue < k0 + n) {
+              s_region[ue - k0] = rp + e * P;
+              s_ux[ue - k0] = ((xs[e >> 1] >> (16 * (e & 1))) & 0xffffu) | ((uint32_t)slot << 16);
             }
           }
         }
-      };
-      // the first kRingEarly stages, then (x cache released) the rest of the prologue
-#pragma unroll 1
-      for (int st = 0; st < kRingEarly; ++st) {
-        if (st < n_stages) issue(st);
-        cp_async_commit();
-      }
-      if (outputs_pending) write_outputs();  // while the first copies are in flight
-      __syncthreads();                       // nobody reads the x cache any more
-      xc_valid = false;
-#pragma unroll 1
-      for (int st = kRingEarly; st < kRing - 1; ++st) {
-        if (st < n_stages) issue(st);
-        cp_async_commit();
-      }
-
-      // B fragments per k-step: lane (fg, tq) holds B[2tq, 2tq+1][fg] and B[2tq+8, 2tq+9][fg];
-      // B[k][col] = x'' of unit k if the unit's group slot is col, else 0
-      for (int q = tid; q < n_steps * 32; q += kThreads) {
-        const int kk = q >> 5, L = q & 31, col = L >> 2, t2i = 2 * (L & 3);
-        const uint32_t *ux = s_ux + kk * kK;
-        auto bh = [&](uint32_t e) -> uint32_t { return ((int)(e >> 16) == col) ? (e & 0xffffu) : 0u; };
-        s_bfrag[q] = make_uint2(bh(ux[t2i]) | (bh(ux[t2i + 1]) << 16),
-                                bh(ux[t2i + 8]) | (bh(ux[t2i + 9]) << 16));
-      }
-
-      float d[8][4];
-#pragma unroll
-      for (int bk = 0; bk < 8; ++bk) d[bk][0] = d[bk][1] = d[bk][2] = d[bk][3] = 0.0f;
-
-      for (int st = 0; st < n_stages; ++st) {
-        cp_async_wait<kRing - 2>();  // this thread's copies of stage st (and s/z) landed
-        __syncthreads();             // everybody's; and stage st-1 is no longer read
-        if (st + kRing - 1 < n_stages) issue(st + kRing - 1);
-        cp_async_commit();
-        const uint32_t *sb = ring + (size_t)(st % kRing) * (kStage * kRow);
-        // this warp's k-steps of the stage: h = kp and kp + 2; operands of both first
-        uint32_t wv[2][4];
-        uint2 bv[2];
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-          const int h = kp + 2 * i, kk = kStage / kK * st + h;
-          const uint32_t *pw = sb + (h * kK + 2 * tq) * kRow + 8 * ob + fg;
-          wv[i][0] = pw[0];
-          wv[i][1] = pw[kRow];
-          wv[i][2] = pw[8 * kRow];
-          wv[i][3] = pw[9 * kRow];
-          bv[i] = s_bfrag[min(kk, n_steps - 1) * 32 + lane];
+        for (int k = n + tid; k < n_pad; k += kThreads) {  // padding units: no load, B = 0
+          s_region[k] = -1;
+          s_ux[k] = 0u;
         }
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-          const int kk = kStage / kK * st + kp + 2 * i;
-          if (kk < n_steps) {
-            const uint32_t w0 = wv[i][0], w1 = wv[i][1], w2 = wv[i][2], w3 = wv[i][3];
-            const uint2 bb = bv[i];
-            // m0/m1: outputs 0-7 / 8-15 of units 2tq (low half) and 2tq+1 (high half);
-            // m2/m3: the same for units 2tq+8 and 2tq+9; nX = mX >> 6 for t' >= 5
-            const uint32_t m0 = prmt(w0, w1, 0x5410u), m1 = prmt(w0, w1, 0x7632u);
-            const uint32_t m2 = prmt(w2, w3, 0x5410u), m3 = prmt(w2, w3, 0x7632u);
-            const uint32_t n0 = m0 >> 6, n1 = m1 >> 6, n2 = m2 >> 6, n3 = m3 >> 6;
-            constexpr uint32_t F = 0x00030003u;
-            // block bk: rows fg (output t = 2bk) and fg+8 (t = 2bk+1) of word fg
-            mma16816(d[0], m0 & (F << 0), m0 & (F << 2), m2 & (F << 0), m2 & (F << 2), bb.x, bb.y);
-            mma16816(d[1], m0 & (F << 4), m0 & (F << 6), m2 & (F << 4), m2 & (F << 6), bb.x, bb.y);
-            mma16816(d[2], m0 & (F << 8), n0 & (F << 4), m2 & (F << 8), n2 & (F << 4), bb.x, bb.y);
-            mma16816(d[3], n0 & (F << 6), n0 & (F << 8), n2 & (F << 6), n2 & (F << 8), bb.x, bb.y);
-            mma16816(d[4], m1 & (F << 0), m1 & (F << 2), m3 & (F << 0), m3 & (F << 2), bb.x, bb.y);
-            mma16816(d[5], m1 & (F << 4), m1 & (F << 6), m3 & (F << 4), m3 & (F << 6), bb.x, bb.y);
-            mma16816(d[6], m1 & (F << 8), n1 & (F << 4), m3 & (F << 8), n3 & (F << 4), bb.x, bb.y);
-            mma16816(d[7], n1 & (F << 6), n1 & (F << 8), n3 & (F << 6), n3 & (F << 8), bb.x, bb.y);
-          }
-        }
-      }
-      cp_async_wait<0>();
+        __syncthreads();
 
-      // flush: y_t += s (D 2^(24 - pos(t) + c) [+ Phi]) [+ z X] for the lane's two slots
+        // ring: stage st holds units 64 st .. 64 st + 63 of the round
+        auto issue = [&](int st) {
+          uint32_t *dst_stage = ring + (size_t)(st % kRing) * (kStage * kRow);
 #pragma unroll
-      for (int jj = 0; jj < 2; ++jj) {
-        const int j = 2 * tq + jj;
-        if (j < ng) {
-          const SlotInfo si = s_slot[j];
-          const uint16_t *srow = s_st + j * kTile + 128 * ob + 16 * fg;
-          const uint16_t *zrow = z_st + j * kTile + 128 * ob + 16 * fg;
-          float sv[16], zv[16];
-          const uint4 s0 = *reinterpret_cast<const uint4 *>(srow);
-          const uint4 s1 = *reinterpret_cast<const uint4 *>(srow + 8);
-          const uint4 z0 = *reinterpret_cast<const uint4 *>(zrow);
-          const uint4 z1 = *reinterpret_cast<const uint4 *>(zrow + 8);
-          const uint32_t su[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
-          const uint32_t zu[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
+          for (int h = 0; h < 2; ++h) {
+            const int q = tid + h * kThreads, ul = q >> 4, part16 = q & 15;
+            const int k = st * kStage + ul;
+            const int region = k < n_pad ? s_region[k] : -1;
+            const int word = wbase + part16 * 4;
+            uint32_t *dst = dst_stage + ul * kRow + part16 * 4;
+            if (region >= 0) {
+              const uint32_t *src = a.planes + (size_t)region * a.W + word;
+              if (ALIGNED) {
+                if (word < a.W) cp_async16(dst, src, 16);
+              } else {
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const float2 fs = __half22float2(*reinterpret_cast<const __half2 *>(&su[k]));
-            const float2 fz = __half22float2(*reinterpret_cast<const __half2 *>(&zu[k]));
-            sv[2 * k] = fs.x;
-            sv[2 * k + 1] = fs.y;
-            zv[2 * k] = fz.x;
-            zv[2 * k + 1] = fz.y;
-          }
-#pragma unroll
-          for (int bk = 0; bk < 8; ++bk) {
-            const int t0 = 2 * bk, t1 = 2 * bk + 1;
-            float v0 = d[bk][jj] * exp2i(24 - field_pos(t0) + si.c);
-            float v1 = d[bk][2 + jj] * exp2i(24 - field_pos(t1) + si.c);
-            if (si.first && kp == 0) {
-              v0 += si.Phi;
-              v1 += si.Phi;
-              yacc[t0] = fmaf(zv[t0], si.X, yacc[t0]);
-              yacc[t1] = fmaf(zv[t1], si.X, yacc[t1]);
+                for (int v = 0; v < 4; ++v)
+                  if (word + v < a.W) cp_async4(dst + v, src + v);
+              }
             }
-            yacc[t0] = fmaf(sv[t0], v0, yacc[t0]);
-            yacc[t1] = fmaf(sv[t1], v1, yacc[t1]);
+          }
+        };
+        // the first kRingEarly stages, then (x cache released) the rest of the prologue
+#pragma unroll
+        for (int st = 0; st < kRingEarly; ++st) {
+          if (st < n_stages) issue(st);
+          cp_async_commit();
+        }
+        if (xc_valid) {
+          __syncthreads();  // nobody reads the x cache any more
+          xc_valid = false;
+        }
+#pragma unroll
+        for (int st = kRingEarly; st < kRing - 1; ++st) {
+          if (st < n_stages) issue(st);
+          cp_async_commit();
+        }
+
+        // B fragments per k-step: lane (fg, tq) holds B[2tq, 2tq+1][fg] and B[2tq+8, 2tq+9][fg];
+        // B[k][col] = x'' of unit k if the unit's group slot is col, else 0
+        for (int q = tid; q < n_steps * 32; q += kThreads) {
+          const int kk = q >> 5, L = q & 31, col = L >> 2, t2i = 2 * (L & 3);
+          const uint32_t *ux = s_ux + kk * kK;
+          auto bh = [&](uint32_t e) -> uint32_t { return ((int)(e >> 16) == col) ? (e & 0xffffu) : 0u; };
+          s_bfrag[q] = make_uint2(bh(ux[t2i]) | (bh(ux[t2i + 1]) << 16),
+                                  bh(ux[t2i + 8]) | (bh(ux[t2i + 9]) << 16));
+        }
+
+        float d[8][4];
+#pragma unroll
+        for (int bk = 0; bk < 8; ++bk) d[bk][0] = d[bk][1] = d[bk][2] = d[bk][3] = 0.0f;
+
+        for (int st = 0; st < n_stages; ++st) {
+          cp_async_wait<kRing - 2>();  // this thread's copies of stage st (and s/z) landed
+          __syncthreads();             // everybody's; and stage st-1 is no longer read
+          if (st + kRing - 1 < n_stages) issue(st + kRing - 1);
+          cp_async_commit();
+          const uint32_t *sb = ring + (size_t)(st % kRing) * (kStage * kRow);
+          // this warp's k-steps of the stage: h = kp and kp + 2; operands of both first
+          uint32_t wv[2][4];
+          uint2 bv[2];
+#pragma unroll
+          for (int i = 0; i < 2; ++i) {
+            const int h = kp + 2 * i, kk = kStage / kK * st + h;
+            const uint32_t *pw = sb + (h * kK + 2 * tq) * kRow + 8 * ob + fg;
+            wv[i][0] = pw[0];
+            wv[i][1] = pw[kRow];
+            wv[i][2] = pw[8 * kRow];
+            wv[i][3] = pw[9 * kRow];
+            bv[i] = s_bfrag[min(kk, n_steps - 1) * 32 + lane];
+          }
+#pragma unroll
+          for (int i = 0; i < 2; ++i) {
+            const int kk = kStage / kK * st + kp + 2 * i;
+            if (kk < n_steps) {
+              const uint32_t w0 = wv[i][0], w1 = wv[i][1], w2 = wv[i][2], w3 = wv[i][3];
+              const uint2 bb = bv[i];
+              // m0/m1: outputs 0-7 / 8-15 of units 2tq (low half) and 2tq+1 (high half);
+              // m2/m3: the same for units 2tq+8 and 2tq+9; nX = mX >> 6 for t' >= 5
+              const uint32_t m0 = prmt(w0, w1, 0x5410u), m1 = prmt(w0, w1, 0x7632u);
+              const uint32_t m2 = prmt(w2, w3, 0x5410u), m3 = prmt(w2, w3, 0x7632u);
+              const uint32_t n0 = m0 >> 6, n1 = m1 >> 6, n2 = m2 >> 6, n3 = m3 >> 6;
+              constexpr uint32_t F = 0x00030003u;
+              // block bk: rows fg (output t = 2bk) and fg+8 (t = 2bk+1) of word fg
+              mma16816(d[0], m0 & (F << 0), m0 & (F << 2), m2 & (F << 0), m2 & (F << 2), bb.x, bb.y);
+              mma16816(d[1], m0 & (F << 4), m0 & (F << 6), m2 & (F << 4), m2 & (F << 6), bb.x, bb.y);
+              mma16816(d[2], m0 & (F << 8), n0 & (F << 4), m2 & (F << 8), n2 & (F << 4), bb.x, bb.y);
+              mma16816(d[3], n0 & (F << 6), n0 & (F << 8), n2 & (F << 6), n2 & (F << 8), bb.x, bb.y);
+              mma16816(d[4], m1 & (F << 0), m1 & (F << 2), m3 & (F << 0), m3 & (F << 2), bb.x, bb.y);
+              mma16816(d[5], m1 & (F << 4), m1 & (F << 6), m3 & (F << 4), m3 & (F << 6), bb.x, bb.y);
+              mma16816(d[6], m1 & (F << 8), n1 & (F << 4), m3 & (F << 8), n3 & (F << 4), bb.x, bb.y);
+              mma16816(d[7], n1 & (F << 6), n1 & (F << 8), n3 & (F << 6), n3 & (F << 8), bb.x, bb.y);
+            }
+          }
+        }
+        cp_async_wait<0>();
+
+        // flush: y_t += s (D 2^(24 - pos(t) + c) [+ Phi]) [+ z X] for the lane's two slots;
+        // the slice's group terms once per window (first round, even-k warps)
+        const bool terms = k0 == 0 && kp == 0;
+#pragma unroll
+        for (int jj = 0; jj < 2; ++jj) {
+          const int j = 2 * tq + jj;
+          if (j < ng) {
+            const SlotInfo si = s_slot[j];
+            const uint16_t *srow = s_st + j * kTile + 128 * ob + 16 * fg;
+            const uint16_t *zrow = z_st + j * kTile + 128 * ob + 16 * fg;
+            float sv[16], zv[16];
+            const uint4 s0 = *reinterpret_cast<const uint4 *>(srow);
+            const uint4 s1 = *reinterpret_cast<const uint4 *>(srow + 8);
+            const uint4 z0 = *reinterpret_cast<const uint4 *>(zrow);
+            const uint4 z1 = *reinterpret_cast<const uint4 *>(zrow + 8);
+            const uint32_t su[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+            const uint32_t zu[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+              const float2 fs = __half22float2(*reinterpret_cast<const __half2 *>(&su[k]));
+              const float2 fz = __half22float2(*reinterpret_cast<const __half2 *>(&zu[k]));
+              sv[2 * k] = fs.x;
+              sv[2 * k + 1] = fs.y;
+              zv[2 * k] = fz.x;
+              zv[2 * k + 1] = fz.y;
+            }
+#pragma unroll
+            for (int bk = 0; bk < 8; ++bk) {
+              const int t0 = 2 * bk, t1 = 2 * bk + 1;
+              float v0 = d[bk][jj] * exp2i(24 - field_pos(t0) + si.c);
+              float v1 = d[bk][2 + jj] * exp2i(24 - field_pos(t1) + si.c);
+              if (terms) {
+                v0 += si.Phi;
+                v1 += si.Phi;
+                yacc[t0] = fmaf(zv[t0], si.X, yacc[t0]);
+                yacc[t1] = fmaf(zv[t1], si.X, yacc[t1]);
+              }
+              yacc[t0] = fmaf(sv[t0], v0, yacc[t0]);
+              yacc[t1] = fmaf(sv[t1], v1, yacc[t1]);
+            }
           }
         }
       }
@@ -614,6 +632,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
     const int ol = 128 * ob + 16 * fg + 8 * (tq & 1) + 4 * (tq >> 1);  // first of 4 outputs
     const int obase = tile * kTile;
     // odd-k warps hand their sums to the even-k warp of the same block
+    __syncthreads();  // s_red of the previous tile is consumed
     if (kp == 1) *reinterpret_cast<float4 *>(s_red + ol) = make_float4(fin[0], fin[1], fin[2], fin[3]);
     __syncthreads();
     if (kp == 0) {
@@ -641,29 +660,26 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
       s_last = atomicInc(&a.counters[tile], (unsigned)(m - 1)) == (unsigned)(m - 1);
     }
     __syncthreads();
-    if (s_last && tid < kTile / 4) {
+    if (s_last) {
+      static_assert(2 * kThreads == kTile, "two outputs per thread");
       __threadfence();
       const int c_first = tile * m;
-      float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-      const float *src = a.partials + (size_t)c_first * kTile + 4 * tid;
-      for (int c0 = 0; c0 < m; c0 += 16) {
-        float4 v[16];
+      float2 acc = make_float2(0.0f, 0.0f);
+      const float *src = a.partials + (size_t)c_first * kTile + 2 * tid;
+      for (int c0 = 0; c0 < m; c0 += 24) {
+        float2 v[24];
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-          v[i] = (c0 + i < m) ? __ldcg(reinterpret_cast<const float4 *>(src + (size_t)(c0 + i) * kTile))
-                              : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        for (int i = 0; i < 24; ++i)
+          v[i] = (c0 + i < m) ? __ldcg(reinterpret_cast<const float2 *>(src + (size_t)(c0 + i) * kTile))
+                              : make_float2(0.0f, 0.0f);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
+        for (int i = 0; i < 24; ++i) {
           acc.x += v[i].x;
           acc.y += v[i].y;
-          acc.z += v[i].z;
-          acc.w += v[i].w;
         }
       }
-      const float out[4] = {acc.x, acc.y, acc.z, acc.w};
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-        if (obase + 4 * tid + i < a.d_out) a.y[obase + 4 * tid + i] = out[i];
+      if (obase + 2 * tid < a.d_out) a.y[obase + 2 * tid] = acc.x;
+      if (obase + 2 * tid + 1 < a.d_out) a.y[obase + 2 * tid + 1] = acc.y;
     }
   }
 }
