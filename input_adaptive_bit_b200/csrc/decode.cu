@@ -84,8 +84,8 @@ static_assert(kSmRing % 16 == 0 && kSmX % 16 == 0 && kSmS % 16 == 0 && kSmZ % 16
                   kSmBfrag % 16 == 0 && kSmLoff % 16 == 0 && kSmSlot % 16 == 0 &&
                   kSmWsum % 16 == 0 && kSmRed % 16 == 0,
               "16-byte aligned regions");
-static_assert(kStage * 16 == 2 * kThreads, "two 16-byte copies per thread and stage");
-static_assert(kStage == 4 * kK && kWarps == 2 * kBlocks, "two k-steps per warp and stage");
+static_assert((kStage * 16) % kThreads == 0, "whole 16-byte copies per thread and stage");
+static_assert(kStage % (2 * kK) == 0 && kWarps == 2 * kBlocks, "k-steps split between two warps");
 static_assert(kMaxG == kThreads, "one group per thread in the output CTAs' scan");
 
 struct SlotInfo {
@@ -302,6 +302,23 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
   const int C = gridDim.x, c = blockIdx.x;
   const int P = a.P;
 
+  // ---- what depends on the shapes only: computed before the wait below, so it
+  // overlaps the tail of the kernel launched before (programmatic launch) ----
+  // the last CTAs write the optional outputs, the others run the GEMV; they are
+  // set aside whether or not outputs are asked for, so y does not depend on it
+  const int n_out = C > 2 * kOutCtas ? kOutCtas : 1;
+  const int C_g = C - n_out;
+  // tiles x row slices: m CTAs per tile, CTA `part` takes the 8-row chunks
+  // [R8 part / m, R8 (part + 1) / m); more tiles than CTAs: whole tiles in turn
+  const bool many = a.tiles >= C_g;
+  const int m = many ? 1 : C_g / a.tiles;
+  const int C_eff = many ? C_g : a.tiles * m;
+  const int R8 = a.d_in / 8;
+  const int part = many ? 0 : c % m;
+  const int q_lo = R8 * part / m, q_hi = R8 * (part + 1) / m;  // R8 <= 2^13, part < 2^8
+  const int row_lo = 8 * q_lo, row_hi = 8 * q_hi;
+  const int tile_first = many ? c : c / m, tile_step = many ? C_g : a.tiles;
+
   // x, theta and the weights may be written by the kernel launched just before
   asm volatile("griddepcontrol.wait;\n" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
@@ -318,10 +335,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
     }
   };
 
-  // the last CTAs write the optional outputs, the others run the GEMV; they are
-  // set aside whether or not outputs are asked for, so y does not depend on it
-  const int n_out = C > 2 * kOutCtas ? kOutCtas : 1;
-  const int C_g = C - n_out;
   if (c >= C_g) {
     if (a.b || a.lists || a.counts || a.grp_sums) {
       load_thresholds();
@@ -331,16 +344,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
   }
   bool thresholds_loaded = false;
 
-  // tiles x row slices: m CTAs per tile, CTA `part` takes the 8-row chunks
-  // [R8 part / m, R8 (part + 1) / m); more tiles than CTAs: whole tiles in turn
-  const bool many = a.tiles >= C_g;
-  const int m = many ? 1 : C_g / a.tiles;
-  const int C_eff = many ? C_g : a.tiles * m;
   if (c >= C_eff) return;
-  const int R8 = a.d_in / 8;
-  const int part = many ? 0 : c % m;
-  const int q_lo = R8 * part / m, q_hi = R8 * (part + 1) / m;  // R8 <= 2^13, part < 2^8
-  const int row_lo = 8 * q_lo, row_hi = 8 * q_hi;
 
   // the slice of x to shared memory when it fits (else it is read from global memory)
   bool xc_valid = row_hi - row_lo <= kXCache;
@@ -348,7 +352,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
     for (int q = tid; q < q_hi - q_lo; q += kThreads) cp_async16(xc + 8 * q, a.x + row_lo + 8 * q, 16);
   cp_async_commit();
 
-  for (int tile = many ? c : c / m; tile < a.tiles; tile += many ? C_g : a.tiles) {
+  for (int tile = tile_first; tile < a.tiles; tile += tile_step) {
     const int wbase = tile * kTileW;  // first word of the tile in a plane region
     float yacc[16];
 #pragma unroll
@@ -428,14 +432,20 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
         }
       }
       __syncthreads();
-      int base = 0, Nw = 0;
+      // exclusive prefix of the 32 (slot, plane) totals, one per lane, by shuffles
+      int base, Nw;
+      {
+        static_assert(4 * kSlots == 32, "one (slot, plane) total per lane");
+        const int t = s_tot[lane];
+        int inc = t;
 #pragma unroll
-      for (int j = 0; j < 4 * kSlots; ++j) {
-        const int t = s_tot[j];
-        base += (j < 4 * slot + pl) ? t : 0;
-        Nw += t;
+        for (int off = 1; off < 32; off <<= 1) {
+          const int u = __shfl_up_sync(0xffffffffu, inc, off);
+          if (lane >= off) inc += u;
+        }
+        Nw = __shfl_sync(0xffffffffu, inc, 31);
+        base = __shfl_sync(0xffffffffu, inc - t, 4 * slot + pl) + (int)pre;  // this thread's first unit
       }
-      base += (int)pre;  // this thread's first unit in the window
       // x 4^(P-1-pl) 2^-c of the thread's 8 rows, rounded to fp16 (a power-of-two
       // product: exact unless the result is subnormal, then rounded as fp16 does)
       uint32_t xs[4] = {0u, 0u, 0u, 0u};
@@ -472,11 +482,69 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
         }
         __syncthreads();
 
-        // ring: stage st holds units 64 st .. 64 st + 63 of the round
+        // B fragments per k-step: lane (fg, tq) holds B[2tq, 2tq+1][fg] and B[2tq+8, 2tq+9][fg];
+        // B[k][col] = x'' of unit k if the unit's group slot is col, else 0
+        auto build_bfrag = [&]() {
+          for (int q = tid; q < n_steps * 32; q += kThreads) {
+            const int kk = q >> 5, L = q & 31, col = L >> 2, t2i = 2 * (L & 3);
+            const uint32_t *ux = s_ux + kk * kK;
+            auto bh = [&](uint32_t e) -> uint32_t { return ((int)(e >> 16) == col) ? (e & 0xffffu) : 0u; };
+            s_bfrag[q] = make_uint2(bh(ux[t2i]) | (bh(ux[t2i + 1]) << 16),
+                                    bh(ux[t2i + 8]) | (bh(ux[t2i + 9]) << 16));
+          }
+        };
+
+        float d[8][4];
+#pragma unroll
+        for (int bk = 0; bk < 8; ++bk) d[bk][0] = d[bk][1] = d[bk][2] = d[bk][3] = 0.0f;
+
+        // this warp's MMA work on ring stage st (units 64 st .. 64 st + 63 of the round,
+        // held in `sb`): its k-steps h = kp and kp + 2, operands of both first
+        constexpr int kStepsPerWarp = kStage / kK / 2;  // k-steps of a stage per warp
+        auto compute = [&](const uint32_t *sb, int st) {
+          uint32_t wv[kStepsPerWarp][4];
+          uint2 bv[kStepsPerWarp];
+#pragma unroll
+          for (int i = 0; i < kStepsPerWarp; ++i) {
+            const int h = kp + 2 * i, kk = kStage / kK * st + h;
+            const uint32_t *pw = sb + (h * kK + 2 * tq) * kRow + 8 * ob + fg;
+            wv[i][0] = pw[0];
+            wv[i][1] = pw[kRow];
+            wv[i][2] = pw[8 * kRow];
+            wv[i][3] = pw[9 * kRow];
+            bv[i] = s_bfrag[min(kk, n_steps - 1) * 32 + lane];
+          }
+#pragma unroll
+          for (int i = 0; i < kStepsPerWarp; ++i) {
+            const int kk = kStage / kK * st + kp + 2 * i;
+            if (kk < n_steps) {
+              const uint32_t w0 = wv[i][0], w1 = wv[i][1], w2 = wv[i][2], w3 = wv[i][3];
+              const uint2 bb = bv[i];
+              // m0/m1: outputs 0-7 / 8-15 of units 2tq (low half) and 2tq+1 (high half);
+              // m2/m3: the same for units 2tq+8 and 2tq+9; nX = mX >> 6 for t' >= 5
+              const uint32_t m0 = prmt(w0, w1, 0x5410u), m1 = prmt(w0, w1, 0x7632u);
+              const uint32_t m2 = prmt(w2, w3, 0x5410u), m3 = prmt(w2, w3, 0x7632u);
+              const uint32_t n0 = m0 >> 6, n1 = m1 >> 6, n2 = m2 >> 6, n3 = m3 >> 6;
+              constexpr uint32_t F = 0x00030003u;
+              // block bk: rows fg (output t = 2bk) and fg+8 (t = 2bk+1) of word fg
+              mma16816(d[0], m0 & (F << 0), m0 & (F << 2), m2 & (F << 0), m2 & (F << 2), bb.x, bb.y);
+              mma16816(d[1], m0 & (F << 4), m0 & (F << 6), m2 & (F << 4), m2 & (F << 6), bb.x, bb.y);
+              mma16816(d[2], m0 & (F << 8), n0 & (F << 4), m2 & (F << 8), n2 & (F << 4), bb.x, bb.y);
+              mma16816(d[3], n0 & (F << 6), n0 & (F << 8), n2 & (F << 6), n2 & (F << 8), bb.x, bb.y);
+              mma16816(d[4], m1 & (F << 0), m1 & (F << 2), m3 & (F << 0), m3 & (F << 2), bb.x, bb.y);
+              mma16816(d[5], m1 & (F << 4), m1 & (F << 6), m3 & (F << 4), m3 & (F << 6), bb.x, bb.y);
+              mma16816(d[6], m1 & (F << 8), n1 & (F << 4), m3 & (F << 8), n3 & (F << 4), bb.x, bb.y);
+              mma16816(d[7], n1 & (F << 6), n1 & (F << 8), n3 & (F << 6), n3 & (F << 8), bb.x, bb.y);
+            }
+          }
+        };
+
+        // ---- cp.async ring: 16 threads copy a unit's segment (16-byte copies; 4-byte
+        // copies for layouts whose rows are not 16-byte aligned) ----
         auto issue = [&](int st) {
           uint32_t *dst_stage = ring + (size_t)(st % kRing) * (kStage * kRow);
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
+          for (int h = 0; h < kStage * 16 / kThreads; ++h) {
             const int q = tid + h * kThreads, ul = q >> 4, part16 = q & 15;
             const int k = st * kStage + ul;
             const int region = k < n_pad ? s_region[k] : -1;
@@ -509,63 +577,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
           if (st < n_stages) issue(st);
           cp_async_commit();
         }
-
-        // B fragments per k-step: lane (fg, tq) holds B[2tq, 2tq+1][fg] and B[2tq+8, 2tq+9][fg];
-        // B[k][col] = x'' of unit k if the unit's group slot is col, else 0
-        for (int q = tid; q < n_steps * 32; q += kThreads) {
-          const int kk = q >> 5, L = q & 31, col = L >> 2, t2i = 2 * (L & 3);
-          const uint32_t *ux = s_ux + kk * kK;
-          auto bh = [&](uint32_t e) -> uint32_t { return ((int)(e >> 16) == col) ? (e & 0xffffu) : 0u; };
-          s_bfrag[q] = make_uint2(bh(ux[t2i]) | (bh(ux[t2i + 1]) << 16),
-                                  bh(ux[t2i + 8]) | (bh(ux[t2i + 9]) << 16));
-        }
-
-        float d[8][4];
-#pragma unroll
-        for (int bk = 0; bk < 8; ++bk) d[bk][0] = d[bk][1] = d[bk][2] = d[bk][3] = 0.0f;
-
+        build_bfrag();
         for (int st = 0; st < n_stages; ++st) {
           cp_async_wait<kRing - 2>();  // this thread's copies of stage st (and s/z) landed
           __syncthreads();             // everybody's; and stage st-1 is no longer read
           if (st + kRing - 1 < n_stages) issue(st + kRing - 1);
           cp_async_commit();
-          const uint32_t *sb = ring + (size_t)(st % kRing) * (kStage * kRow);
-          // this warp's k-steps of the stage: h = kp and kp + 2; operands of both first
-          uint32_t wv[2][4];
-          uint2 bv[2];
-#pragma unroll
-          for (int i = 0; i < 2; ++i) {
-            const int h = kp + 2 * i, kk = kStage / kK * st + h;
-            const uint32_t *pw = sb + (h * kK + 2 * tq) * kRow + 8 * ob + fg;
-            wv[i][0] = pw[0];
-            wv[i][1] = pw[kRow];
-            wv[i][2] = pw[8 * kRow];
-            wv[i][3] = pw[9 * kRow];
-            bv[i] = s_bfrag[min(kk, n_steps - 1) * 32 + lane];
-          }
-#pragma unroll
-          for (int i = 0; i < 2; ++i) {
-            const int kk = kStage / kK * st + kp + 2 * i;
-            if (kk < n_steps) {
-              const uint32_t w0 = wv[i][0], w1 = wv[i][1], w2 = wv[i][2], w3 = wv[i][3];
-              const uint2 bb = bv[i];
-              // m0/m1: outputs 0-7 / 8-15 of units 2tq (low half) and 2tq+1 (high half);
-              // m2/m3: the same for units 2tq+8 and 2tq+9; nX = mX >> 6 for t' >= 5
-              const uint32_t m0 = prmt(w0, w1, 0x5410u), m1 = prmt(w0, w1, 0x7632u);
-              const uint32_t m2 = prmt(w2, w3, 0x5410u), m3 = prmt(w2, w3, 0x7632u);
-              const uint32_t n0 = m0 >> 6, n1 = m1 >> 6, n2 = m2 >> 6, n3 = m3 >> 6;
-              constexpr uint32_t F = 0x00030003u;
-              // block bk: rows fg (output t = 2bk) and fg+8 (t = 2bk+1) of word fg
-              mma16816(d[0], m0 & (F << 0), m0 & (F << 2), m2 & (F << 0), m2 & (F << 2), bb.x, bb.y);
-              mma16816(d[1], m0 & (F << 4), m0 & (F << 6), m2 & (F << 4), m2 & (F << 6), bb.x, bb.y);
-              mma16816(d[2], m0 & (F << 8), n0 & (F << 4), m2 & (F << 8), n2 & (F << 4), bb.x, bb.y);
-              mma16816(d[3], n0 & (F << 6), n0 & (F << 8), n2 & (F << 6), n2 & (F << 8), bb.x, bb.y);
-              mma16816(d[4], m1 & (F << 0), m1 & (F << 2), m3 & (F << 0), m3 & (F << 2), bb.x, bb.y);
-              mma16816(d[5], m1 & (F << 4), m1 & (F << 6), m3 & (F << 4), m3 & (F << 6), bb.x, bb.y);
-              mma16816(d[6], m1 & (F << 8), n1 & (F << 4), m3 & (F << 8), n3 & (F << 4), bb.x, bb.y);
-              mma16816(d[7], n1 & (F << 6), n1 & (F << 8), n3 & (F << 6), n3 & (F << 8), bb.x, bb.y);
-            }
-          }
+          compute(ring + (size_t)(st % kRing) * (kStage * kRow), st);
         }
         cp_async_wait<0>();
 
