@@ -54,6 +54,8 @@ FALLBACK_HBM_GBS = 6650.0
 NCU_TRAFFIC = {
     # gemv.cu, grinqh_gemv (profiles/grinqh_gemv_qwen3-8b-proj_launches.md)
     "84585736bc0dc9cf2ac9f0a4738586346a63ac0a4e44acbdc753bb3917df6db4": 17150844,
+    # decode.cu, grinqh_decode_gemv (profiles/decode_kernel_qwen3-8b-proj_launches.md)
+    "d2de23db3e7b387068aa504a680887d244caf606d2e45789fcd05cc32ebda22d": 17111019,
 }
 KERNEL_SOURCE = {"fused": "decode.cu", "two": "gemv.cu"}
 
