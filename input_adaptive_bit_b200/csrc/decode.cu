@@ -51,7 +51,7 @@ constexpr int kRow = kTileW + 4;      // shared words per unit row: conflict-fre
 constexpr int kK = 16;                // units per MMA k-step
 constexpr int kStage = 64;            // units per ring stage (4 k-steps, 2 per warp)
 constexpr int kRing = 8;              // ring stages
-constexpr int kRingEarly = 6;         // stages issued before the x cache (on the last slots) is freed
+constexpr int kXSlot = 6;             // first ring slot that holds the x cache in the front end
 constexpr int kRound = 1024;          // units per round
 constexpr int kSlots = 8;             // groups per window (the MMA n dimension)
 constexpr int kMaxG = kDecodeMaxDin / kGroup;
@@ -62,8 +62,8 @@ constexpr int kOutCtas = 4;           // CTAs that write the optional outputs
 // shared memory map (bytes)
 constexpr size_t kStageBytes = (size_t)kStage * kRow * 4;
 constexpr size_t kSmRing = 0;                                               // u32 [kRing][kStage][kRow]
-constexpr size_t kSmX = kSmRing + (size_t)kRingEarly * kStageBytes;         // fp16 [kXCache], aliases
-                                                                            // ring slots >= kRingEarly
+constexpr size_t kSmX = kSmRing + (size_t)kXSlot * kStageBytes;             // fp16 [kXCache], aliases
+                                                                            // ring slots >= kXSlot
 constexpr size_t kSmRegion = kSmRing + (size_t)kRing * kStageBytes;         // i32 [kRound]
 constexpr size_t kSmUx = kSmRegion + kRound * 4;                            // u32 [kRound]: xh | slot << 16
 constexpr size_t kSmBfrag = kSmUx + kRound * 4;                             // uint2 [kRound / kK][32]
@@ -78,7 +78,7 @@ constexpr size_t kSmCnt = kSmRing;                                          // u
 constexpr size_t kSmLoff = kSmCnt + (size_t)kMaxG * 4;                      // int4 [kMaxG]: list offsets
 constexpr size_t kSmWsum = kSmLoff + (size_t)kMaxG * 16;                    // int4 [kWarps]
 static_assert(kSmBytes <= 227 * 1024, "shared memory");
-static_assert((size_t)kXCache * 2 <= (size_t)(kRing - kRingEarly) * kStageBytes, "x cache fits");
+static_assert((size_t)kXCache * 2 <= (size_t)(kRing - kXSlot) * kStageBytes, "x cache fits");
 static_assert(kSmWsum + kWarps * 16 <= kSmX, "output-CTA arrays below the x cache");
 static_assert(kSmRing % 16 == 0 && kSmX % 16 == 0 && kSmS % 16 == 0 && kSmZ % 16 == 0 &&
                   kSmBfrag % 16 == 0 && kSmLoff % 16 == 0 && kSmSlot % 16 == 0 &&
@@ -562,18 +562,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
             }
           }
         };
-        // the first kRingEarly stages, then (x cache released) the rest of the prologue
+        // the prologue (the x cache on the last ring slots was last read before the
+        // barrier above, so its slots are free)
+        xc_valid = false;
 #pragma unroll
-        for (int st = 0; st < kRingEarly; ++st) {
-          if (st < n_stages) issue(st);
-          cp_async_commit();
-        }
-        if (xc_valid) {
-          __syncthreads();  // nobody reads the x cache any more
-          xc_valid = false;
-        }
-#pragma unroll
-        for (int st = kRingEarly; st < kRing - 1; ++st) {
+        for (int st = 0; st < kRing - 1; ++st) {
           if (st < n_stages) issue(st);
           cp_async_commit();
         }
