@@ -409,6 +409,21 @@ def oracle_sample_run(spec, rank=0, seconds=10.0, outs_per_rep=None):
 
 # ---- main ------------------------------------------------------------------------------
 
+def max_over_ranks(dist, v: float, device) -> float:
+    """The largest v over all ranks (v itself without a process group)."""
+    if dist is None:
+        return v
+    import torch
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_gbps(world: int, bytes_per_rank: float, ms: float) -> float:
+    """Weak scaling: every rank moved bytes_per_rank in at most ms (the max over ranks)."""
+    return world * bytes_per_rank / (ms * 1e-3) / 1e9
+
+
 def dist_env():
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -488,12 +503,6 @@ def main(argv=None):
         if dist is not None:
             dist.barrier()
 
-    def max_over_ranks(v):
-        if dist is None:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
 
     # warm-up
     with torch.cuda.stream(wl.stream):
@@ -510,9 +519,9 @@ def main(argv=None):
     barrier()
     time.sleep(0.1)
     clocks = ClockSampler.summarize(sampler.stop())
-    ms = max_over_ranks(ms)
+    ms = max_over_ranks(dist, ms, device)
     bytes_timed = sum(step_bytes[i % N_POOL] for i in range(args.steps))
-    value = world * bytes_timed / (ms * 1e-3) / 1e9
+    value = whole_job_gbps(world, bytes_timed, ms)
     n_gemv = len(specs)
 
     # ---- the dominant kernel -------------------------------------------------------
@@ -523,8 +532,8 @@ def main(argv=None):
         wl.two_graph.replay()
         ms_g = device_time_ms(torch, wl.stream, lambda i: wl.gemv_graph.replay(), reps)
         ms_two = device_time_ms(torch, wl.stream, lambda i: wl.two_graph.replay(), reps)
-    ms_g = max_over_ranks(ms_g)
-    ms_two = max_over_ranks(ms_two)
+    ms_g = max_over_ranks(dist, ms_g, device)
+    ms_two = max_over_ranks(dist, ms_two, device)
     gemv_launch_us = ms_g * 1e3 / (reps * n_gemv)
     peak, peak_kind = measured_peaks()
     if args.path == "fused":
@@ -560,9 +569,9 @@ def main(argv=None):
         t0 = time.perf_counter()
         ms_e2e = device_time_ms(torch, wl.stream, e2e_step, k_e2e)
         wall_e2e = (time.perf_counter() - t0) * 1e3
-    ms_e2e = max_over_ranks(max(ms_e2e, wall_e2e))
+    ms_e2e = max_over_ranks(dist, max(ms_e2e, wall_e2e), device)
     e2e_bytes = sum(step_bytes[i % N_POOL] for i in range(k_e2e))
-    e2e_value = world * e2e_bytes / (ms_e2e * 1e-3) / 1e9
+    e2e_value = whole_job_gbps(world, e2e_bytes, ms_e2e)
 
     cases = None
     dense4 = None
