@@ -136,8 +136,7 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
 // D += A B, m16n8k16, fp16 operands, fp32 accumulators.
 __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                          uint32_t a3, uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
       "{%8,%9}, {%0,%1,%2,%3};\n"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
@@ -460,8 +459,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
       }
 
       for (int k0 = 0; k0 < Nw; k0 += kRound) {
-        const int n = min(kRound, Nw - k0), n_pad = (n + kK - 1) & ~(kK - 1);
-        const int n_steps = n_pad / kK, n_stages = (n_pad + kStage - 1) / kStage;
+        // the round is padded to whole stages with units whose B entries are 0 and
+        // which load nothing: every warp runs every k-step of a stage unconditionally
+        const int n = min(kRound, Nw - k0), n_pad = (n + kStage - 1) & ~(kStage - 1);
+        const int n_steps = n_pad / kK, n_stages = n_pad / kStage;
+        static_assert(kRound % kStage == 0, "rounds of whole stages");
         if (k0 > 0) __syncthreads();  // the previous round no longer reads the records
 
         // this thread's units that fall in [k0, k0 + n)
@@ -512,12 +514,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
             wv[i][1] = pw[kRow];
             wv[i][2] = pw[8 * kRow];
             wv[i][3] = pw[9 * kRow];
-            bv[i] = s_bfrag[min(kk, n_steps - 1) * 32 + lane];
+            bv[i] = s_bfrag[kk * 32 + lane];
           }
 #pragma unroll
           for (int i = 0; i < kStepsPerWarp; ++i) {
-            const int kk = kStage / kK * st + kp + 2 * i;
-            if (kk < n_steps) {
+            {
               const uint32_t w0 = wv[i][0], w1 = wv[i][1], w2 = wv[i][2], w3 = wv[i][3];
               const uint2 bb = bv[i];
               // m0/m1: outputs 0-7 / 8-15 of units 2tq (low half) and 2tq+1 (high half);
