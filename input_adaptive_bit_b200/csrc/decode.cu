@@ -382,23 +382,25 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
       cp_async_wait<1>();  // the x slice (committed before) has landed
       __syncthreads();
 
-      // compaction: a 16-thread team per (group slot, plane); thread gsub of team
-      // (slot, pl) takes chunk 16 (g_w + slot) + gsub of the window and that
-      // chunk's units of plane pl.  Units are placed slot by slot, then plane by
-      // plane, then chunk by chunk, then row by row (the order within a round is free)
+      // compaction: a 16-thread team per (plane, group slot); thread gsub of team
+      // (pl, slot) takes chunk 16 (g_w + slot) + gsub of the window and that
+      // chunk's units of plane pl.  The plane-0 teams (warps 0-3) also take the
+      // slot's B-column scale and group sums.  Units are placed slot by slot, then
+      // plane by plane, then chunk by chunk, then row by row (the order within a
+      // round is free)
       static_assert(kSlots * 4 * kGT == kThreads, "one team per slot and plane");
-      const int slot = tid >> 6, pl = (tid >> 4) & 3;
+      const int pl = tid / (kSlots * kGT), slot = (tid / kGT) % kSlots;
       const int qc = kGT * (g_w + slot) + gsub;  // the thread's chunk
       const bool act = qc >= q_lo && qc < q_hi;
       uint4 xw = make_uint4(0, 0, 0, 0);
-      uint32_t mk[4] = {0u, 0u, 0u, 0u};
-      if (act) {
+      if (act)
         xw = xc_valid ? *reinterpret_cast<const uint4 *>(xc + 8 * (qc - q_lo))
                       : __ldg(reinterpret_cast<const uint4 *>(a.x + 8 * qc));
-        plane_masks8(xw, t2, P, mk);
-      }
-      int cg;
-      {
+      uint32_t mp = 0u;  // this team's plane mask of the chunk
+      if (pl == 0) {     // warps 0-3
+        uint32_t mk[4] = {0u, 0u, 0u, 0u};
+        if (act) plane_masks8(xw, t2, P, mk);
+        mp = mk[0];
         // B-column scale: the largest active |x| of the slot times 4^(P-1) stays below 2^16
         const uint32_t w[4] = {xw.x, xw.y, xw.z, xw.w};
         uint32_t amax = 0;
@@ -407,9 +409,19 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
           if ((mk[0] >> e) & 1u) amax = max(amax, (w[e >> 1] >> (16 * (e & 1))) & 0x7fffu);
 #pragma unroll
         for (int off = 8; off > 0; off >>= 1) amax = max(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-        cg = (amax >= 0x7c00u) ? 0 : max(0, (int)(amax >> 10) - 15 + 2 * P - 16);
+        float X, Phi;
+        group_sums8(xw, mk, phi, X, Phi);
+        if (gsub == 0) {
+          SlotInfo si = {(amax >= 0x7c00u) ? 0 : max(0, (int)(amax >> 10) - 15 + 2 * P - 16), X,
+                         Phi, 0};
+          s_slot[slot] = si;
+        }
+      } else if (act && pl < P) {
+        __half2 tp = t2[3];
+        if (pl == 1) tp = t2[1];
+        if (pl == 2) tp = t2[2];
+        mp = plane_mask8(xw, tp);
       }
-      const uint32_t mp = pl == 0 ? mk[0] : pl == 1 ? mk[1] : pl == 2 ? mk[2] : mk[3];
       const uint32_t cnt = (uint32_t)__popc(mp);
       uint32_t pre;
       {
@@ -421,14 +433,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
         }
         pre = inc - cnt;
         if (gsub == kGT - 1) s_tot[4 * slot + pl] = (int)inc;
-      }
-      if ((warp & 1) == 0) {  // the warps holding planes 0 and 1: the slot's group sums
-        float X, Phi;
-        group_sums8(xw, mk, phi, X, Phi);
-        if (pl == 0 && gsub == 0) {
-          SlotInfo si = {cg, X, Phi, 0};
-          s_slot[slot] = si;
-        }
       }
       __syncthreads();
       // exclusive prefix of the 32 (slot, plane) totals, one per lane, by shuffles
@@ -447,6 +451,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
       }
       // x 4^(P-1-pl) 2^-c of the thread's 8 rows, rounded to fp16 (a power-of-two
       // product: exact unless the result is subnormal, then rounded as fp16 does)
+      const int cg = s_slot[slot].c;
       uint32_t xs[4] = {0u, 0u, 0u, 0u};
       if (pl < P) {
         const __half2 sc = __half2half2(__ushort_as_half((uint16_t)((15 + 2 * (P - 1 - pl) - cg) << 10)));
@@ -678,14 +683,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
       const int c_first = tile * m;
       float2 acc = make_float2(0.0f, 0.0f);
       const float *src = a.partials + (size_t)c_first * kTile + 2 * tid;
-      for (int c0 = 0; c0 < m; c0 += 24) {
-        float2 v[24];
+      for (int c0 = 0; c0 < m; c0 += 40) {  // one L2 round trip for up to 40 partials
+        float2 v[40];
 #pragma unroll
-        for (int i = 0; i < 24; ++i)
+        for (int i = 0; i < 40; ++i)
           v[i] = (c0 + i < m) ? __ldcg(reinterpret_cast<const float2 *>(src + (size_t)(c0 + i) * kTile))
                               : make_float2(0.0f, 0.0f);
 #pragma unroll
-        for (int i = 0; i < 24; ++i) {
+        for (int i = 0; i < 40; ++i) {
           acc.x += v[i].x;
           acc.y += v[i].y;
         }

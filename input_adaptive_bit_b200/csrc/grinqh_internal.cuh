@@ -109,6 +109,17 @@ __device__ __forceinline__ void plane_masks8(uint4 xw, const __half2 (&t2)[4], i
   }
 }
 
+// The mask of one plane: bit e = (row e has b > 2p), t = that plane's threshold.
+__device__ __forceinline__ uint32_t plane_mask8(uint4 xw, __half2 t) {
+  const uint32_t w[4] = {xw.x & 0x7fff7fffu, xw.y & 0x7fff7fffu, xw.z & 0x7fff7fffu,
+                         xw.w & 0x7fff7fffu};
+  uint32_t v = 0;
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+    v |= (__hge2_mask(*reinterpret_cast<const __half2 *>(&w[j]), t) & 0x00010001u) << (2 * j);
+  return (v | (v >> 15)) & 0xFFu;
+}
+
 // Level (b/2) of row e from its plane masks.
 __device__ __forceinline__ int row_level(const uint32_t (&mask)[4], int e) {
   return (int)(((mask[0] >> e) & 1u) + ((mask[1] >> e) & 1u) + ((mask[2] >> e) & 1u) +
