@@ -305,55 +305,92 @@ def device_time_ms(torch, stream, fn, n):
     return e0.elapsed_time(e1)
 
 
-def cold_case_times(wl, reps=20):
-    """Per-GEMV device time with a cold L2 (a 256 MB write before every launch):
-    the fused decode call, assign + gemv, and gemv alone."""
-    torch = wl.torch
-    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=wl.device)
-    rows = []
-    st = wl.stream
+class L2Flush:
+    """Evicts the L2 by reading a 256 MB buffer (written once): the L2 is left
+    holding clean lines, so the timed launch pays no write-back of a flush."""
+
+    def __init__(self, torch, device):
+        self.buf = torch.ones(256 * 1024 * 1024 // 4, dtype=torch.float32, device=device)
+        self.sink = torch.empty(1, dtype=torch.float32, device=device)
+
+    def __call__(self):
+        self.sink.copy_(self.buf.sum().reshape(1))
+
+
+def _graph_ms(torch, st, body, reps):
+    """Mean device ms of one replay of a graph that runs body() `reps` times."""
     with torch.cuda.stream(st):
-        for j, (lin, spec) in enumerate(zip(wl.layers[:16], wl.specs[:16])):
-            t = {"fused": [], "all": [], "gemv": []}
-            for r in range(reps):
-                k = r % N_POOL
-                for mode in t:
-                    flush.fill_(float(r))
-                    if mode == "gemv":
-                        lin.assign(wl.xv(k, j), wl.thetas[j], stream=st)
-                        flush.fill_(float(r) + 0.5)
-                    e0 = torch.cuda.Event(enable_timing=True)
-                    e1 = torch.cuda.Event(enable_timing=True)
-                    e0.record(st)
-                    if mode == "fused":
-                        lin.decode(wl.xv(k, j), wl.thetas[j], y=wl.yv(j), stream=st)
-                    else:
-                        if mode == "all":
-                            lin.assign(wl.xv(k, j), wl.thetas[j], stream=st)
-                        lin.gemv(wl.yv(j), stream=st)
-                    e1.record(st)
-                    e1.synchronize()
-                    t[mode].append(e0.elapsed_time(e1) * 1e3)
-            b = lin.b.cpu().numpy()
-            med = {m: statistics.median(v) for m, v in t.items()}
-            rows.append({"name": spec.name, "d_in": spec.d_in, "d_out": spec.d_out,
-                         "b_max": spec.b_max, "eff_bits": round(float(b.mean()), 3),
-                         "us_fused": round(med["fused"], 2),
-                         "fused_GBps": round(min_bytes(b, spec.d_out) / (med["fused"] * 1e3), 1),
-                         "us_assign_gemv": round(med["all"], 2),
-                         "us_gemv": round(med["gemv"], 2),
-                         "gemv_GBps": round(min_bytes(b, spec.d_out, False)
-                                            / (med["gemv"] * 1e3), 1)})
+        body()  # warm-up (first launches, smem attributes)
+        st.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=st):
+            for _ in range(reps):
+                body()
+        g.replay()
+        st.synchronize()
+        ms = device_time_ms(torch, st, lambda i: g.replay(), 5)
+    del g
+    return ms / 5
+
+
+def cold_case_times(wl, reps=20):
+    """Per-GEMV device time with a cold L2: a graph of reps x (256 MB read, call)
+    minus a graph of reps x (256 MB read), per call -- the fused decode call,
+    assign + gemv, and gemv alone after an untimed assign."""
+    torch = wl.torch
+    flush = L2Flush(torch, wl.device)
+    st = wl.stream
+    t_flush = _graph_ms(torch, st, flush, reps) / reps
+    rows = []
+    for j, (lin, spec) in enumerate(zip(wl.layers[:16], wl.specs[:16])):
+        xj, thj, yj = wl.xv(0, j), wl.thetas[j], wl.yv(j)
+
+        def fused():
+            flush()
+            lin.decode(xj, thj, y=yj, stream=st)
+
+        def two():
+            flush()
+            lin.assign(xj, thj, stream=st)
+            lin.gemv(yj, stream=st)
+
+        def assign_only():
+            flush()
+            lin.assign(xj, thj, stream=st)
+            flush()
+
+        def gemv_after_assign():
+            flush()
+            lin.assign(xj, thj, stream=st)
+            flush()
+            lin.gemv(yj, stream=st)
+
+        med = {"fused": _graph_ms(torch, st, fused, reps) / reps - t_flush,
+               "all": _graph_ms(torch, st, two, reps) / reps - t_flush,
+               # both graphs hold the same two reads and assign: the difference is gemv
+               "gemv": (_graph_ms(torch, st, gemv_after_assign, reps)
+                        - _graph_ms(torch, st, assign_only, reps)) / reps}
+        med = {k: v * 1e3 for k, v in med.items()}  # us
+        b = lin.b.cpu().numpy()
+        rows.append({"name": spec.name, "d_in": spec.d_in, "d_out": spec.d_out,
+                     "b_max": spec.b_max, "eff_bits": round(float(b.mean()), 3),
+                     "us_fused": round(med["fused"], 2),
+                     "fused_GBps": round(min_bytes(b, spec.d_out) / (med["fused"] * 1e3), 1),
+                     "us_assign_gemv": round(med["all"], 2),
+                     "us_gemv": round(med["gemv"], 2),
+                     "gemv_GBps": round(min_bytes(b, spec.d_out, False) / (med["gemv"] * 1e3), 1)})
     return rows
 
 
 def dense4_times(wl, reps=20):
-    """The in-library dense 4-bit comparator on each distinct shape, cold L2."""
+    """The in-library dense 4-bit comparator on each distinct shape, cold L2
+    (graph of reps x (256 MB read, call) minus the reads)."""
     torch = wl.torch
     from input_adaptive_bit_b200.layer import Dense4Linear
-    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=wl.device)
-    seen, rows = set(), []
+    flush = L2Flush(torch, wl.device)
     st = wl.stream
+    t_flush = _graph_ms(torch, st, flush, reps) / reps
+    seen, rows = set(), []
     for j, spec in enumerate(wl.specs[:16]):
         if (spec.d_in, spec.d_out) in seen:
             continue
@@ -361,23 +398,33 @@ def dense4_times(wl, reps=20):
         g = synth.rng(spec.config_id, 5000 + j, 0)
         q4, s, z = synth.rtn_quantize(synth.gaussian_weights(g, spec.d_in, spec.d_out), 4)
         d4 = Dense4Linear(q4, s, z, device=wl.device)
-        ts = []
-        with torch.cuda.stream(st):
-            for r in range(reps):
-                flush.fill_(float(r))
-                e0 = torch.cuda.Event(enable_timing=True)
-                e1 = torch.cuda.Event(enable_timing=True)
-                e0.record(st)
-                d4(wl.xv(r % N_POOL, j), stream=st)
-                e1.record(st)
-                e1.synchronize()
-                ts.append(e0.elapsed_time(e1) * 1e3)
-        t = statistics.median(ts)
+        xj = wl.xv(0, j)
+
+        def call():
+            flush()
+            d4(xj, stream=st)
+
+        t = (_graph_ms(torch, st, call, reps) / reps - t_flush) * 1e3
         nbytes = spec.d_in * spec.d_out // 2 + 4 * spec.d_out * (spec.d_in // 128) + 4 * spec.d_out
         rows.append({"name": f"dense4_{spec.d_in}x{spec.d_out}", "us": round(t, 2),
                      "GBps": round(nbytes / (t * 1e3), 1)})
         del d4
     return rows
+
+
+def bits_fit(cases, specs):
+    """Least-squares fit of fused latency against bits over the uniform-width
+    cases (b_max 8): slope (us per bit), intercept and R^2."""
+    pts = [(spec.uniform_b, c["us_fused"]) for c, spec in zip(cases, specs)
+           if spec.uniform_b is not None and spec.b_max == 8]
+    if len(pts) < 3:
+        return None
+    b = np.array([p[0] for p in pts], np.float64)
+    t = np.array([p[1] for p in pts], np.float64)
+    c, a = np.polyfit(b, t, 1)
+    r2 = 1.0 - float(np.sum((t - (a + c * b)) ** 2)) / float(np.sum((t - t.mean()) ** 2))
+    return {"us_per_bit": round(float(c), 3), "us_at_0_bits": round(float(a), 3),
+            "r2": round(r2, 4), "points": [[int(x), round(float(y), 2)] for x, y in pts]}
 
 
 # ---- the oracle on the host cores (baseline only) --------------------------------
@@ -626,6 +673,9 @@ def main(argv=None):
     if cases is not None:
         line["cases"] = cases
         line["dense4"] = dense4
+        fit = bits_fit(cases, specs)
+        if fit is not None:
+            line["latency_vs_bits"] = fit
     print(json.dumps(line), flush=True)
     return 0
 
