@@ -322,17 +322,18 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
   asm volatile("griddepcontrol.wait;\n" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
 
-  // thresholds and phi (loaded where their latency hides behind copies in flight)
-  __half2 t2[4];
-  float phi[5];
-  auto load_thresholds = [&]() {
-    make_thresholds(a.theta, P, t2);
+  // thresholds and phi: loaded first (their latency hides behind the copies
+  // issued next), sorted and converted where they are first needed
+  float th_raw[4], phi[5];
 #pragma unroll
-    for (int k = 0; k <= 4; ++k) {
-      const float def = (2 * k < a.b_max) ? exp2i(a.b_max - 2 * k - 1) : 0.0f;
-      phi[k] = (k <= P) ? (a.phi ? a.phi[k] : def) : 0.0f;
-    }
-  };
+  for (int k = 0; k < 4; ++k) th_raw[k] = (k < P) ? a.theta[k] : __int_as_float(0x7fc00000);
+#pragma unroll
+  for (int k = 0; k <= 4; ++k) {
+    const float def = (2 * k < a.b_max) ? exp2i(a.b_max - 2 * k - 1) : 0.0f;
+    phi[k] = (k <= P) ? (a.phi ? a.phi[k] : def) : 0.0f;
+  }
+  __half2 t2[4];
+  auto load_thresholds = [&]() { sort_thresholds(th_raw, t2); };
 
   if (c >= C_g) {
     if (a.b || a.lists || a.counts || a.grp_sums) {
@@ -360,7 +361,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
     // windows of kSlots groups over the slice
     for (int g_w = row_lo / kGroup; g_w * kGroup < row_hi; g_w += kSlots) {
       const int ng = min(kSlots, (row_hi + kGroup - 1) / kGroup - g_w);
-      __syncthreads();  // the previous window no longer reads the staged data
+      if (g_w != row_lo / kGroup || tile != tile_first)
+        __syncthreads();  // the previous window no longer reads the staged data
 
       // stage s and z rows of the window's groups for this tile (past d_out: zero)
 #pragma unroll
@@ -396,30 +398,34 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
       if (act)
         xw = xc_valid ? *reinterpret_cast<const uint4 *>(xc + 8 * (qc - q_lo))
                       : __ldg(reinterpret_cast<const uint4 *>(a.x + 8 * qc));
-      uint32_t mp = 0u;  // this team's plane mask of the chunk
-      if (pl == 0) {     // warps 0-3
+      // this team's plane mask of the chunk; the plane-1 warps also take the slot's
+      // group sums, the plane-2 warps its B-column scale (in parallel)
+      uint32_t mp = 0u;
+      if (pl == 1) {  // warps 4-7
         uint32_t mk[4] = {0u, 0u, 0u, 0u};
         if (act) plane_masks8(xw, t2, P, mk);
-        mp = mk[0];
-        // B-column scale: the largest active |x| of the slot times 4^(P-1) stays below 2^16
+        mp = mk[1];
+        float X, Phi;
+        group_sums8(xw, mk, phi, X, Phi);
+        if (gsub == 0) {
+          s_slot[slot].X = X;
+          s_slot[slot].Phi = Phi;
+        }
+      } else if (pl == 2) {  // warps 8-11
+        // the largest active |x| of the slot, times 4^(P-1), stays below 2^16
+        const uint32_t m0 = act ? plane_mask8(xw, t2[0]) : 0u;
+        if (act && P > 2) mp = plane_mask8(xw, t2[2]);
         const uint32_t w[4] = {xw.x, xw.y, xw.z, xw.w};
         uint32_t amax = 0;
 #pragma unroll
         for (int e = 0; e < 8; ++e)
-          if ((mk[0] >> e) & 1u) amax = max(amax, (w[e >> 1] >> (16 * (e & 1))) & 0x7fffu);
+          if ((m0 >> e) & 1u) amax = max(amax, (w[e >> 1] >> (16 * (e & 1))) & 0x7fffu);
 #pragma unroll
         for (int off = 8; off > 0; off >>= 1) amax = max(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-        float X, Phi;
-        group_sums8(xw, mk, phi, X, Phi);
-        if (gsub == 0) {
-          SlotInfo si = {(amax >= 0x7c00u) ? 0 : max(0, (int)(amax >> 10) - 15 + 2 * P - 16), X,
-                         Phi, 0};
-          s_slot[slot] = si;
-        }
-      } else if (act && pl < P) {
+        if (gsub == 0) s_slot[slot].c = (amax >= 0x7c00u) ? 0 : max(0, (int)(amax >> 10) - 15 + 2 * P - 16);
+      } else if (act && pl < P) {  // warps 0-3 and 12-15
         __half2 tp = t2[3];
-        if (pl == 1) tp = t2[1];
-        if (pl == 2) tp = t2[2];
+        if (pl == 0) tp = t2[0];
         mp = plane_mask8(xw, tp);
       }
       const uint32_t cnt = (uint32_t)__popc(mp);

@@ -72,11 +72,9 @@ inline WsLayout ws_layout(int d_in, int d_out, int b_max) {
 // theta holds exactly when |x_i| >= (theta rounded up to fp16).  So one packed
 // fp16 comparison per two rows and plane gives the plane masks bit-exactly.
 
-// Sorted, fp16-rounded-up thresholds; entries past P (and NaN thresholds) are NaN.
-__device__ __forceinline__ void make_thresholds(const float *theta, int P, __half2 (&t2)[4]) {
-  float th[4];
-#pragma unroll
-  for (int k = 0; k < 4; ++k) th[k] = (k < P) ? theta[k] : __int_as_float(0x7fc00000);
+// Sorted, fp16-rounded-up thresholds from the P raw values in th (entries past P
+// must be NaN, as must NaN thresholds stay): ascending, NaN last.
+__device__ __forceinline__ void sort_thresholds(float (&th)[4], __half2 (&t2)[4]) {
   auto cs = [](float &x, float &y) {
     const bool sw = (x != x) ? (y == y) : (y < x);
     if (sw) {
@@ -92,6 +90,14 @@ __device__ __forceinline__ void make_thresholds(const float *theta, int P, __hal
   cs(th[1], th[2]);
 #pragma unroll
   for (int k = 0; k < 4; ++k) t2[k] = __half2half2(__float2half_ru(th[k]));
+}
+
+// Sorted, fp16-rounded-up thresholds; entries past P (and NaN thresholds) are NaN.
+__device__ __forceinline__ void make_thresholds(const float *theta, int P, __half2 (&t2)[4]) {
+  float th[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) th[k] = (k < P) ? theta[k] : __int_as_float(0x7fc00000);
+  sort_thresholds(th, t2);
 }
 
 // mask[p] bit e = (row e of the 8 rows in xw has b > 2p); rows in memory order.
