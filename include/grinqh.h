@@ -136,7 +136,15 @@ int grinqh_gemv(const uint32_t *planes, const uint16_t *s, const uint16_t *z,
  *                 bytes (zero-filled once; left zeroed), used for the split-K
  *                 partial sums and counters only.
  * Limits: d_in <= 65536 (GRINQH_ERR_UNSUPPORTED_SHAPE otherwise; use
- * grinqh_assign + grinqh_gemv there).  Deterministic. */
+ * grinqh_assign + grinqh_gemv there).  Deterministic.
+ * Launch overlap: the kernel may start while the kernel before it on `stream`
+ * is still finishing (programmatic dependent launch), and it reads theta and
+ * phi before waiting for that kernel; x, planes, s and z are read only after
+ * the wait, and every output is written after it.  So theta and phi must not
+ * be written by the kernel launched immediately before this call on the same
+ * stream (a copy, an event or any other kernel in between lifts this).  The
+ * split-K arrival wait does not give up on a correct launch; if it does (after
+ * about a second) it sets the device error word to 3. */
 int grinqh_decode_gemv(const uint32_t *planes, const uint16_t *s, const uint16_t *z,
                        const uint16_t *x, const float *theta, const float *phi, int d_in,
                        int d_out, int b_max, float *y, uint8_t *b, int32_t *lists,

@@ -13,16 +13,17 @@
 //      A_{g,o} = sum over units (i, p) of group g of x_i 4^(P-1-p) slice_p(i, o),
 //    where a unit is one (row, plane) pair with b_i > 2p and slice_p is the
 //    2-bit field of plane p.  X_g, Phi_g are per-group sums of x and x phi.
-//  * Units are ordered by group, plane, row (the order of the per-plane lists
-//    within a group).  Every CTA derives the whole order itself from x and
-//    theta: it counts each group's units per plane (one warp per group), scans
-//    the counts, and then compacts only the groups its own range touches.  No
-//    other kernel and no global round trip sit between x and the GEMV.
-//  * Work = 1024-output tiles x unit ranges.  A unit's tile segment is 256
-//    contiguous bytes of its plane region.  Each tile's U units are cut into
-//    m = floor(CTAs / tiles) equal contiguous ranges, one per CTA (one wave,
-//    balanced whatever the sparsity); the m partial tiles are added by the
-//    last CTA to arrive, in CTA order (deterministic).
+//  * Work = 1024-output tiles x row slices.  A unit's tile segment is 256
+//    contiguous bytes of its plane region.  Each tile's d_in rows are cut into
+//    m = floor(CTAs / tiles) contiguous slices, one per CTA (one wave); every
+//    CTA derives its own units from x and theta -- one row per lane, a ballot
+//    per plane, a scan of the per-(group, plane, 32-row chunk) counts -- so no
+//    other kernel and no global round trip sit between x and the GEMV.  Units
+//    are ordered by group, plane, row.
+//  * The m partial tiles of a tile meet in global memory: every CTA of the tile
+//    publishes its partial, waits until all m have arrived, and adds up its
+//    own 1/m share of the outputs over the m partials in CTA order
+//    (deterministic).
 //  * A CTA walks its range in rounds of at most 1024 units and 8 groups.  The
 //    segments stream through an 8-stage shared-memory ring (cp.async, 16 B per
 //    thread and copy, one barrier per 32 units).
@@ -51,28 +52,34 @@ constexpr int kRow = kTileW + 4;      // shared words per unit row: conflict-fre
 constexpr int kK = 16;                // units per MMA k-step
 constexpr int kStage = 64;            // units per ring stage (4 k-steps, 2 per warp)
 constexpr int kRing = 8;              // ring stages
-constexpr int kXSlot = 6;             // first ring slot that holds the x cache in the front end
+constexpr int kXSlot = 6;             // first ring slot of the output CTAs' x cache
 constexpr int kRound = 1024;          // units per round
 constexpr int kSlots = 8;             // groups per window (the MMA n dimension)
 constexpr int kMaxG = kDecodeMaxDin / kGroup;
 constexpr int kXCache = 16384;        // rows of x held in shared memory
-constexpr int kGT = 16;               // threads per group: one 8-row chunk each
+constexpr int kGT = 16;               // output CTAs: threads per group, one 8-row chunk each
+constexpr int kChunkRows = 32;        // GEMV front end: rows per warp chunk, one per lane
+constexpr int kSpinLimit = 1 << 20;   // polls of a split-K counter before giving up (about 1 s)
 constexpr int kOutCtas = 4;           // CTAs that write the optional outputs
 
 // shared memory map (bytes)
 constexpr size_t kStageBytes = (size_t)kStage * kRow * 4;
 constexpr size_t kSmRing = 0;                                               // u32 [kRing][kStage][kRow]
-constexpr size_t kSmX = kSmRing + (size_t)kXSlot * kStageBytes;             // fp16 [kXCache], aliases
-                                                                            // ring slots >= kXSlot
+constexpr size_t kSmX = kSmRing + (size_t)kXSlot * kStageBytes;             // fp16 [kXCache] (output
+                                                                            // CTAs), ring slots >= kXSlot
 constexpr size_t kSmRegion = kSmRing + (size_t)kRing * kStageBytes;         // i32 [kRound]
 constexpr size_t kSmUx = kSmRegion + kRound * 4;                            // u32 [kRound]: xh | slot << 16
 constexpr size_t kSmBfrag = kSmUx + kRound * 4;                             // uint2 [kRound / kK][32]
 constexpr size_t kSmS = kSmBfrag + (size_t)(kRound / kK) * 32 * 8;          // fp16 [kSlots][kTile]
 constexpr size_t kSmZ = kSmS + (size_t)kSlots * kTile * 2;                  // fp16 [kSlots][kTile]
 constexpr size_t kSmSlot = kSmZ + (size_t)kSlots * kTile * 2;               // SlotInfo [kSlots]
-constexpr size_t kSmTot = kSmSlot + kSlots * 16;                            // i32 [kSlots][4]: window units
-constexpr size_t kSmRed = kSmTot + kSlots * 16;                             // fp32 [kTile]: odd-k warps
-constexpr size_t kSmBytes = kSmRed + (size_t)kTile * 4;
+constexpr size_t kSmRed = kSmSlot + kSlots * 16;                            // fp32 [kTile]: odd-k warps
+constexpr size_t kSmChunkCnt = kSmRed + (size_t)kTile * 4;                  // i32 [kSlots][4][4]: units per
+                                                                            // (slot, plane, chunk)
+constexpr size_t kSmWarpSum = kSmChunkCnt + kSlots * 4 * 4 * 4;             // float4 [kWarps]: X, Phi, max|x|
+constexpr size_t kSmWarpBal = kSmWarpSum + kWarps * 16;                     // u32 [kWarps][2][4]: ballots
+constexpr size_t kSmWarpOff = kSmWarpBal + kWarps * 32;                     // i32 [kWarps][2][4]: first units
+constexpr size_t kSmBytes = kSmWarpOff + kWarps * 32;
 // the output CTAs keep their counts and scans where the GEMV CTAs have the ring
 constexpr size_t kSmCnt = kSmRing;                                          // u32 [kMaxG]: plane counts, bytes
 constexpr size_t kSmLoff = kSmCnt + (size_t)kMaxG * 4;                      // int4 [kMaxG]: list offsets
@@ -82,11 +89,13 @@ static_assert((size_t)kXCache * 2 <= (size_t)(kRing - kXSlot) * kStageBytes, "x 
 static_assert(kSmWsum + kWarps * 16 <= kSmX, "output-CTA arrays below the x cache");
 static_assert(kSmRing % 16 == 0 && kSmX % 16 == 0 && kSmS % 16 == 0 && kSmZ % 16 == 0 &&
                   kSmBfrag % 16 == 0 && kSmLoff % 16 == 0 && kSmSlot % 16 == 0 &&
-                  kSmWsum % 16 == 0 && kSmRed % 16 == 0,
+                  kSmWsum % 16 == 0 && kSmRed % 16 == 0 && kSmChunkCnt % 16 == 0 &&
+                  kSmWarpSum % 16 == 0 && kSmWarpBal % 16 == 0 && kSmWarpOff % 16 == 0,
               "16-byte aligned regions");
 static_assert((kStage * 16) % kThreads == 0, "whole 16-byte copies per thread and stage");
 static_assert(kStage % (2 * kK) == 0 && kWarps == 2 * kBlocks, "k-steps split between two warps");
 static_assert(kMaxG == kThreads, "one group per thread in the output CTAs' scan");
+static_assert(kGroup == 4 * kChunkRows && kWarps == 2 * kSlots, "two warps per slot, two chunks each");
 
 struct SlotInfo {
   int c;       // the group's B-column scale exponent: B holds x 4^(P-1-p) 2^-c
@@ -110,6 +119,7 @@ struct DecodeArgs {
   float *grp_sums;
   unsigned *counters;
   float *partials;    // [gridDim.x][kTile]
+  int *error;         // the workspace's device error word
 };
 
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
@@ -140,6 +150,12 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
       "{%8,%9}, {%0,%1,%2,%3};\n"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ unsigned ld_acquire(const unsigned *p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];\n" : "=r"(v) : "l"(p) : "memory");
+  return v;
 }
 
 // 2^e as a float, for |e| well inside the normal range.
@@ -282,22 +298,18 @@ template <bool ALIGNED>
 __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
   uint32_t *ring = reinterpret_cast<uint32_t *>(smem + kSmRing);
-  uint16_t *xc = reinterpret_cast<uint16_t *>(smem + kSmX);
   int32_t *s_region = reinterpret_cast<int32_t *>(smem + kSmRegion);
   uint32_t *s_ux = reinterpret_cast<uint32_t *>(smem + kSmUx);
   uint2 *s_bfrag = reinterpret_cast<uint2 *>(smem + kSmBfrag);
   uint16_t *s_st = reinterpret_cast<uint16_t *>(smem + kSmS);
   uint16_t *z_st = reinterpret_cast<uint16_t *>(smem + kSmZ);
   SlotInfo *s_slot = reinterpret_cast<SlotInfo *>(smem + kSmSlot);
-  int *s_tot = reinterpret_cast<int *>(smem + kSmTot);
   float *s_red = reinterpret_cast<float *>(smem + kSmRed);
-  __shared__ int s_last;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int fg = lane >> 2, tq = lane & 3;  // MMA fragment row group and column pair
   const int ob = warp & (kBlocks - 1);      // the warp's 128-output block of the tile
   const int kp = warp / kBlocks;            // ... and its k-step parity
-  const int gsub = tid & (kGT - 1);
   const int C = gridDim.x, c = blockIdx.x;
   const int P = a.P;
 
@@ -317,13 +329,27 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
   const int q_lo = R8 * part / m, q_hi = R8 * (part + 1) / m;  // R8 <= 2^13, part < 2^8
   const int row_lo = 8 * q_lo, row_hi = 8 * q_hi;
   const int tile_first = many ? c : c / m, tile_step = many ? C_g : a.tiles;
+  const int g_first = row_lo / kGroup;
+  auto window_groups = [&](int g_w) { return min(kSlots, (row_hi + kGroup - 1) / kGroup - g_w); };
 
-  // x, theta and the weights may be written by the kernel launched just before
-  asm volatile("griddepcontrol.wait;\n" ::: "memory");
-  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+  // the s and z rows of a window's groups for a tile, to shared memory (past d_out: zero)
+  auto stage_sz = [&](int tile, int g_w, int ng) {
+#pragma unroll
+    for (int i = 0; i < 2 * kSlots * (kTile / 8) / kThreads; ++i) {
+      const int q = tid + i * kThreads;  // [which][slot][chunk of 8 halves]
+      const int which = q / (kSlots * (kTile / 8)), gi = (q / (kTile / 8)) % kSlots;
+      const int ci = q % (kTile / 8), o = tile * kTile + ci * 8;
+      if (gi < ng) {
+        const uint16_t *src = (which ? a.z : a.s) + (size_t)(g_w + gi) * a.d_out + o;
+        uint16_t *dst = (which ? z_st : s_st) + gi * kTile + ci * 8;
+        cp_async16(dst, o < a.d_out ? (const void *)src : (const void *)a.s, o < a.d_out ? 16 : 0);
+      }
+    }
+  };
 
-  // thresholds and phi: loaded first (their latency hides behind the copies
-  // issued next), sorted and converted where they are first needed
+  // ---- theta and phi are not written by the kernel launched just before (a
+  // condition of the call), so they are fetched before waiting for it; x, planes,
+  // s and z only after ----
   float th_raw[4], phi[5];
 #pragma unroll
   for (int k = 0; k < 4; ++k) th_raw[k] = (k < P) ? a.theta[k] : __int_as_float(0x7fc00000);
@@ -332,25 +358,22 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
     const float def = (2 * k < a.b_max) ? exp2i(a.b_max - 2 * k - 1) : 0.0f;
     phi[k] = (k <= P) ? (a.phi ? a.phi[k] : def) : 0.0f;
   }
+  asm volatile("griddepcontrol.wait;\n" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+
   __half2 t2[4];
-  auto load_thresholds = [&]() { sort_thresholds(th_raw, t2); };
+  sort_thresholds(th_raw, t2);
 
   if (c >= C_g) {
-    if (a.b || a.lists || a.counts || a.grp_sums) {
-      load_thresholds();
-      write_outputs(a, smem, c - C_g, n_out, t2, phi);
-    }
+    if (a.b || a.lists || a.counts || a.grp_sums) write_outputs(a, smem, c - C_g, n_out, t2, phi);
     return;
   }
-  bool thresholds_loaded = false;
-
   if (c >= C_eff) return;
 
-  // the slice of x to shared memory when it fits (else it is read from global memory)
-  bool xc_valid = row_hi - row_lo <= kXCache;
-  if (xc_valid)
-    for (int q = tid; q < q_hi - q_lo; q += kThreads) cp_async16(xc + 8 * q, a.x + row_lo + 8 * q, 16);
-  cp_async_commit();
+  int *s_ccnt = reinterpret_cast<int *>(smem + kSmChunkCnt);
+  float4 *s_wsum = reinterpret_cast<float4 *>(smem + kSmWarpSum);
+  uint4 *s_wbal = reinterpret_cast<uint4 *>(smem + kSmWarpBal);
+  int4 *s_woff = reinterpret_cast<int4 *>(smem + kSmWarpOff);
 
   for (int tile = tile_first; tile < a.tiles; tile += tile_step) {
     const int wbase = tile * kTileW;  // first word of the tile in a plane region
@@ -359,93 +382,77 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
     for (int t = 0; t < 16; ++t) yacc[t] = 0.0f;
 
     // windows of kSlots groups over the slice
-    for (int g_w = row_lo / kGroup; g_w * kGroup < row_hi; g_w += kSlots) {
-      const int ng = min(kSlots, (row_hi + kGroup - 1) / kGroup - g_w);
-      if (g_w != row_lo / kGroup || tile != tile_first)
+    for (int g_w = g_first; g_w * kGroup < row_hi; g_w += kSlots) {
+      const int ng = window_groups(g_w);
+      if (g_w != g_first || tile != tile_first)
         __syncthreads();  // the previous window no longer reads the staged data
 
-      // stage s and z rows of the window's groups for this tile (past d_out: zero)
+      // ---- compaction, one row per lane: warp w takes chunks cc = 2 (w mod 2) and
+      // 2 (w mod 2) + 1 (32 rows each) of group slot w / 2, for every plane.  The
+      // window's units are ordered by slot, plane, chunk, row (any order works
+      // within a round: each unit carries its slot into B) ----
+      const int slot = warp >> 1, cc0 = 2 * (warp & 1);
+      const bool live = slot < ng;  // warp-uniform
+      const int row0 = (g_w + slot) * kGroup + kChunkRows * cc0 + lane;  // the lane's row in chunk cc0
+      uint32_t xr = 0u, inb = 0u;  // the lane's two x values (fp16 pair) and which are in the slice
+      uint32_t bal[2][4] = {{0u, 0u, 0u, 0u}, {0u, 0u, 0u, 0u}};
+      if (live) {
 #pragma unroll
-      for (int i = 0; i < 2 * kSlots * (kTile / 8) / kThreads; ++i) {
-        const int q = tid + i * kThreads;  // [which][slot][chunk of 8 halves]
-        const int which = q / (kSlots * (kTile / 8)), gi = (q / (kTile / 8)) % kSlots;
-        const int ci = q % (kTile / 8), o = tile * kTile + ci * 8;
-        if (gi < ng) {
-          const uint16_t *src = (which ? a.z : a.s) + (size_t)(g_w + gi) * a.d_out + o;
-          uint16_t *dst = (which ? z_st : s_st) + gi * kTile + ci * 8;
-          cp_async16(dst, o < a.d_out ? (const void *)src : (const void *)a.s, o < a.d_out ? 16 : 0);
+        for (int ci = 0; ci < 2; ++ci) {
+          const int row = row0 + kChunkRows * ci;
+          if (row >= row_lo && row < row_hi) {
+            xr |= (uint32_t)__ldg(a.x + row) << (16 * ci);
+            inb |= 1u << ci;
+          }
         }
       }
+      // s and z are needed only at the flush: their copies go out after the x loads
+      stage_sz(tile, g_w, ng);
       cp_async_commit();
-      if (!thresholds_loaded) {
-        load_thresholds();
-        thresholds_loaded = true;
+      if (live) {
+        // plane p of a row is loaded when b > 2p, i.e. |x| >= the p-th smallest threshold
+        float X = 0.0f, Phi = 0.0f;
+        uint32_t amax = 0u;
+#pragma unroll
+        for (int ci = 0; ci < 2; ++ci) {
+          const uint32_t xb = (xr >> (16 * ci)) & 0xffffu;
+          const __half ax = __ushort_as_half((uint16_t)(xb & 0x7fffu));
+          int lev = 0;
+#pragma unroll
+          for (int p = 0; p < 4; ++p) {
+            const bool act = ((inb >> ci) & 1u) && __hge(ax, __low2half(t2[p]));
+            bal[ci][p] = __ballot_sync(0xffffffffu, act);
+            lev += act ? 1 : 0;
+          }
+          if (lev > 0) {
+            const float xv = __half2float(__ushort_as_half((uint16_t)xb));
+            X += xv;
+            Phi = __fmaf_rn(xv, pick_phi(phi, lev), Phi);
+            amax = max(amax, xb & 0x7fffu);
+          }
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+          X += __shfl_xor_sync(0xffffffffu, X, off);
+          Phi += __shfl_xor_sync(0xffffffffu, Phi, off);
+        }
+        amax = __reduce_max_sync(0xffffffffu, amax);
+        if (lane == 0) s_wsum[warp] = make_float4(X, Phi, __uint_as_float(amax), 0.0f);
       }
-      cp_async_wait<1>();  // the x slice (committed before) has landed
+      // units per (slot, plane, chunk); lanes 0-7 write the warp's eight
+#pragma unroll
+      for (int ci = 0; ci < 2; ++ci)
+#pragma unroll
+        for (int p = 0; p < 4; ++p)
+          if (lane == 4 * ci + p) s_ccnt[(4 * slot + p) * 4 + cc0 + ci] = __popc(bal[ci][p]);
       __syncthreads();
 
-      // compaction: a 16-thread team per (plane, group slot); thread gsub of team
-      // (pl, slot) takes chunk 16 (g_w + slot) + gsub of the window and that
-      // chunk's units of plane pl.  The plane-0 teams (warps 0-3) also take the
-      // slot's B-column scale and group sums.  Units are placed slot by slot, then
-      // plane by plane, then chunk by chunk, then row by row (the order within a
-      // round is free)
-      static_assert(kSlots * 4 * kGT == kThreads, "one team per slot and plane");
-      const int pl = tid / (kSlots * kGT), slot = (tid / kGT) % kSlots;
-      const int qc = kGT * (g_w + slot) + gsub;  // the thread's chunk
-      const bool act = qc >= q_lo && qc < q_hi;
-      uint4 xw = make_uint4(0, 0, 0, 0);
-      if (act)
-        xw = xc_valid ? *reinterpret_cast<const uint4 *>(xc + 8 * (qc - q_lo))
-                      : __ldg(reinterpret_cast<const uint4 *>(a.x + 8 * qc));
-      // this team's plane mask of the chunk; the plane-1 warps also take the slot's
-      // group sums, the plane-2 warps its B-column scale (in parallel)
-      uint32_t mp = 0u;
-      if (pl == 1) {  // warps 4-7
-        uint32_t mk[4] = {0u, 0u, 0u, 0u};
-        if (act) plane_masks8(xw, t2, P, mk);
-        mp = mk[1];
-        float X, Phi;
-        group_sums8(xw, mk, phi, X, Phi);
-        if (gsub == 0) {
-          s_slot[slot].X = X;
-          s_slot[slot].Phi = Phi;
-        }
-      } else if (pl == 2) {  // warps 8-11
-        // the largest active |x| of the slot, times 4^(P-1), stays below 2^16
-        const uint32_t m0 = act ? plane_mask8(xw, t2[0]) : 0u;
-        if (act && P > 2) mp = plane_mask8(xw, t2[2]);
-        const uint32_t w[4] = {xw.x, xw.y, xw.z, xw.w};
-        uint32_t amax = 0;
-#pragma unroll
-        for (int e = 0; e < 8; ++e)
-          if ((m0 >> e) & 1u) amax = max(amax, (w[e >> 1] >> (16 * (e & 1))) & 0x7fffu);
-#pragma unroll
-        for (int off = 8; off > 0; off >>= 1) amax = max(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-        if (gsub == 0) s_slot[slot].c = (amax >= 0x7c00u) ? 0 : max(0, (int)(amax >> 10) - 15 + 2 * P - 16);
-      } else if (act && pl < P) {  // warps 0-3 and 12-15
-        __half2 tp = t2[3];
-        if (pl == 0) tp = t2[0];
-        mp = plane_mask8(xw, tp);
-      }
-      const uint32_t cnt = (uint32_t)__popc(mp);
-      uint32_t pre;
+      // exclusive prefix over the (slot, plane, chunk) counts: lane L holds the four
+      // chunks of (slot, plane) = (L / 4, L mod 4)
+      int Nw;
       {
-        uint32_t inc = cnt;
-#pragma unroll
-        for (int off = 1; off < kGT; off <<= 1) {
-          const uint32_t t = __shfl_up_sync(0xffffffffu, inc, off, kGT);
-          if (gsub >= off) inc += t;
-        }
-        pre = inc - cnt;
-        if (gsub == kGT - 1) s_tot[4 * slot + pl] = (int)inc;
-      }
-      __syncthreads();
-      // exclusive prefix of the 32 (slot, plane) totals, one per lane, by shuffles
-      int base, Nw;
-      {
-        static_assert(4 * kSlots == 32, "one (slot, plane) total per lane");
-        const int t = s_tot[lane];
+        const int4 cv = reinterpret_cast<const int4 *>(s_ccnt)[lane];
+        const int t = cv.x + cv.y + cv.z + cv.w;
         int inc = t;
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
@@ -453,21 +460,39 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
           if (lane >= off) inc += u;
         }
         Nw = __shfl_sync(0xffffffffu, inc, 31);
-        base = __shfl_sync(0xffffffffu, inc - t, 4 * slot + pl) + (int)pre;  // this thread's first unit
-      }
-      // x 4^(P-1-pl) 2^-c of the thread's 8 rows, rounded to fp16 (a power-of-two
-      // product: exact unless the result is subnormal, then rounded as fp16 does)
-      const int cg = s_slot[slot].c;
-      uint32_t xs[4] = {0u, 0u, 0u, 0u};
-      if (pl < P) {
-        const __half2 sc = __half2half2(__ushort_as_half((uint16_t)((15 + 2 * (P - 1 - pl) - cg) << 10)));
-        const uint32_t w[4] = {xw.x, xw.y, xw.z, xw.w};
+        // first units of chunks cc0 and cc0 + 1 of the lane's (slot, plane)
+        const int o0 = inc - t + (cc0 ? cv.x + cv.y : 0);
+        const int o1 = o0 + (cc0 ? cv.z : cv.x);
+        int offv[2][4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const __half2 r = __hmul2(*reinterpret_cast<const __half2 *>(&w[j]), sc);
-          xs[j] = *reinterpret_cast<const uint32_t *>(&r);
+        for (int p = 0; p < 4; ++p) {
+          offv[0][p] = __shfl_sync(0xffffffffu, o0, 4 * slot + p);
+          offv[1][p] = __shfl_sync(0xffffffffu, o1, 4 * slot + p);
+        }
+        if (live && lane == 0) {
+          s_wbal[2 * warp] = make_uint4(bal[0][0], bal[0][1], bal[0][2], bal[0][3]);
+          s_wbal[2 * warp + 1] = make_uint4(bal[1][0], bal[1][1], bal[1][2], bal[1][3]);
+          s_woff[2 * warp] = make_int4(offv[0][0], offv[0][1], offv[0][2], offv[0][3]);
+          s_woff[2 * warp + 1] = make_int4(offv[1][0], offv[1][1], offv[1][2], offv[1][3]);
         }
       }
+      // the slot's B-column scale exponent: the largest active |x| of the slot, times
+      // 4^(P-1), stays below 2^16; and its group sums (for the flush)
+      int cg = 0;
+      if (live) {
+        const float4 w0 = s_wsum[2 * slot], w1 = s_wsum[2 * slot + 1];
+        const uint32_t am = max(__float_as_uint(w0.z), __float_as_uint(w1.z));
+        cg = (am >= 0x7c00u) ? 0 : max(0, (int)(am >> 10) - 15 + 2 * P - 16);
+        if (cc0 == 0 && lane == 0) {
+          SlotInfo si;
+          si.c = cg;
+          si.X = w0.x + w1.x;
+          si.Phi = w0.y + w1.y;
+          si.pad = 0;
+          s_slot[slot] = si;
+        }
+      }
+      __syncwarp();
 
       for (int k0 = 0; k0 < Nw; k0 += kRound) {
         // the round is padded to whole stages with units whose B entries are 0 and
@@ -477,15 +502,27 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
         static_assert(kRound % kStage == 0, "rounds of whole stages");
         if (k0 > 0) __syncthreads();  // the previous round no longer reads the records
 
-        // this thread's units that fall in [k0, k0 + n)
-        if (cnt > 0) {
-          const int rp = 8 * qc * P + pl;  // region of the chunk's row 0, plane pl
+        // the records of the warp's units that fall in [k0, k0 + n): plane region
+        // and x 4^(P-1-p) 2^-c rounded to fp16 (a power-of-two product: exact unless
+        // the result is subnormal, then rounded as fp16 does) with the slot
+        if (live) {
+          const uint32_t lt = (1u << lane) - 1u;
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const int ue = base + __popc(mp & ((1u << e) - 1u));
-            if (((mp >> e) & 1u) && ue >= k0 && ue < k0 + n) {
-              s_region[ue - k0] = rp + e * P;
-              s_ux[ue - k0] = ((xs[e >> 1] >> (16 * (e & 1))) & 0xffffu) | ((uint32_t)slot << 16);
+          for (int ci = 0; ci < 2; ++ci) {
+            const uint4 bv = s_wbal[2 * warp + ci];
+            const int4 ov = s_woff[2 * warp + ci];
+            const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w};
+            const int ow[4] = {ov.x, ov.y, ov.z, ov.w};
+            const __half xh = __ushort_as_half((uint16_t)((xr >> (16 * ci)) & 0xffffu));
+            const int rp = (row0 + kChunkRows * ci) * P;
+#pragma unroll
+            for (int p = 0; p < 4; ++p) {
+              const int u = ow[p] + __popc(bw[p] & lt);
+              if (((bw[p] >> lane) & 1u) && u >= k0 && u < k0 + n) {
+                const __half sc = __ushort_as_half((uint16_t)((15 + 2 * (P - 1 - p) - cg) << 10));
+                s_region[u - k0] = rp + p;
+                s_ux[u - k0] = (uint32_t)__half_as_ushort(__hmul(xh, sc)) | ((uint32_t)slot << 16);
+              }
             }
           }
         }
@@ -574,9 +611,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
             }
           }
         };
-        // the prologue (the x cache on the last ring slots was last read before the
-        // barrier above, so its slots are free)
-        xc_valid = false;
 #pragma unroll
         for (int st = 0; st < kRing - 1; ++st) {
           if (st < n_stages) issue(st);
@@ -673,36 +707,61 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
       }
       continue;
     }
-    // one of m partial tiles: publish it; the tile's last CTA to arrive adds them
+    // one of m partial tiles: publish it, wait until all m CTAs of the tile have
+    // published theirs, then add up this CTA's share of the tile's outputs
     if (kp == 0)
       *reinterpret_cast<float4 *>(a.partials + (size_t)c * kTile + ol) =
           make_float4(fin[0], fin[1], fin[2], fin[3]);
     __syncthreads();
     if (tid == 0) {
       __threadfence();  // the CTA's partial (ordered before by the barrier) is visible first
-      s_last = atomicInc(&a.counters[tile], (unsigned)(m - 1)) == (unsigned)(m - 1);
+      // the counter counts arrivals modulo m: the tile's last CTA brings it back to 0
+      // (the next call on this workspace waits for this grid to finish before it counts)
+      if (atomicInc(&a.counters[tile], (unsigned)(m - 1)) != (unsigned)(m - 1)) {
+        // every CTA of the grid is resident (one per SM, and the grid that follows
+        // starts only once all of them have started), so the wait ends; the poll
+        // limit only guards against a broken launch
+        int polls = 0;
+        while (ld_acquire(&a.counters[tile]) != 0u) {
+          if (++polls == kSpinLimit) {
+            atomicCAS(a.error, 0, kDevErrSplitKTimeout);
+            break;
+          }
+          __nanosleep(32);
+        }
+      } else {
+        __threadfence();  // the last to arrive: the others' partials are visible to it
+      }
     }
     __syncthreads();
-    if (s_last) {
-      static_assert(2 * kThreads == kTile, "two outputs per thread");
-      __threadfence();
+    {
+      // this CTA's share: quads [Q part / m, Q (part + 1) / m) of the tile's Q = kTile / 4;
+      // m <= kMaxCtas <= Q, so every share is non-empty, and m nq <= Q + m <= kThreads
+      static_assert(kMaxCtas <= kTile / 4 && kTile / 4 + kMaxCtas <= kThreads, "fixup shares");
+      const int q0 = (kTile / 4) * part / m, nq = (kTile / 4) * (part + 1) / m - q0;
       const int c_first = tile * m;
-      float2 acc = make_float2(0.0f, 0.0f);
-      const float *src = a.partials + (size_t)c_first * kTile + 2 * tid;
-      for (int c0 = 0; c0 < m; c0 += 40) {  // one L2 round trip for up to 40 partials
-        float2 v[40];
-#pragma unroll
-        for (int i = 0; i < 40; ++i)
-          v[i] = (c0 + i < m) ? __ldcg(reinterpret_cast<const float2 *>(src + (size_t)(c0 + i) * kTile))
-                              : make_float2(0.0f, 0.0f);
-#pragma unroll
-        for (int i = 0; i < 40; ++i) {
-          acc.x += v[i].x;
-          acc.y += v[i].y;
-        }
+      float4 *s_fix = reinterpret_cast<float4 *>(smem + kSmRing);  // [m][nq]; the ring is idle
+      for (int t = tid; t < m * nq; t += kThreads) {
+        const int cc = t / nq, qq = t - cc * nq;
+        s_fix[t] = __ldcg(reinterpret_cast<const float4 *>(a.partials + (size_t)(c_first + cc) * kTile) +
+                          q0 + qq);
       }
-      if (obase + 2 * tid < a.d_out) a.y[obase + 2 * tid] = acc.x;
-      if (obase + 2 * tid + 1 < a.d_out) a.y[obase + 2 * tid + 1] = acc.y;
+      __syncthreads();
+      if (tid < nq) {
+        float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        for (int cc = 0; cc < m; ++cc) {  // in CTA order: deterministic
+          const float4 v = s_fix[cc * nq + tid];
+          acc.x += v.x;
+          acc.y += v.y;
+          acc.z += v.z;
+          acc.w += v.w;
+        }
+        const int o = obase + 4 * (q0 + tid);
+        if (o < a.d_out) a.y[o] = acc.x;
+        if (o + 1 < a.d_out) a.y[o + 1] = acc.y;
+        if (o + 2 < a.d_out) a.y[o + 2] = acc.z;
+        if (o + 3 < a.d_out) a.y[o + 3] = acc.w;
+      }
     }
   }
 }
@@ -765,6 +824,7 @@ cudaError_t launch_decode(const uint32_t *planes, const uint16_t *s, const uint1
   a.grp_sums = grp_sums;
   a.counters = reinterpret_cast<unsigned *>(w + L.counters);
   a.partials = reinterpret_cast<float *>(w + L.partials);
+  a.error = &reinterpret_cast<WsHeader *>(w)->error;
   cudaError_t e = (a.W % 4 == 0) ? launch_variant<true>(a, st) : launch_variant<false>(a, st);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();

@@ -24,6 +24,7 @@ constexpr int kDecodeMaxDin = 65536;            // largest d_in of the fused dec
 // Device error codes written to the workspace error word.
 constexpr int kDevErrStreamMismatch = 1;  // gemv saw a unit stream of another d_in / b_max
 constexpr int kDevErrBadUnit = 2;         // a unit record outside [0, d_in) x [0, P) (skipped)
+constexpr int kDevErrSplitKTimeout = 3;   // decode: a split-K wait gave up (y of that tile is wrong)
 
 // Workspace header (first 256 bytes of the workspace).
 struct WsHeader {

@@ -1,7 +1,8 @@
 """GPU parity of the fused decode kernel (grinqh_decode_gemv) in the cases its
 own work split creates: ranges spanning several rounds, more tiles than CTAs,
 empty groups between active ones, the largest accepted d_in, fewer units than
-CTAs, and the optional outputs (bit-exact with grinqh_assign, or skipped)."""
+CTAs, every split-K factor from 144 CTAs per tile down to one, and the
+optional outputs (bit-exact with grinqh_assign, or skipped)."""
 import numpy as np
 import pytest
 import torch
@@ -118,3 +119,22 @@ def test_large_activations_use_a_scaled_b_column():
     x = (x.astype(np.float32) * 900.0).clip(-65504, 65504).astype(np.float16)
     theta = theta * np.float32(900.0)
     check_fused(q, s, z, x, theta, 8)
+
+
+@pytest.mark.parametrize("d_out", [1024, 2048, 48 * 1024, 72 * 1024, 144 * 1024])
+def test_split_k_shares_every_ctas_per_tile(d_out):
+    # one tile (every GEMV CTA takes a slice of the same 1024 outputs) down to one
+    # CTA per tile: each CTA of a tile waits for the others and adds its share of
+    # the partial sums; y must be the same on a second call (fixed order) and the
+    # device error word must stay clear
+    from input_adaptive_bit_b200 import grinqh_check_device_error
+    d_in = 512
+    q, s, z, x, theta = cheap_case(8, d_in, d_out, 8)
+    rng = np.random.default_rng(d_out)
+    outs = np.unique(np.concatenate([np.arange(0, 48), np.arange(d_out - 48, d_out),
+                                     rng.integers(0, d_out, 300)])).astype(np.int32)
+    lin, out = check_fused(q, s, z, x, theta, 8, outs=outs)
+    y2 = lin.decode(to_dev(x), to_dev(theta), outputs=False)
+    torch.cuda.synchronize()
+    assert np.array_equal(y2.cpu().numpy().astype(np.float64), out["y"])
+    grinqh_check_device_error(lin.ws)  # raises if a split-K wait gave up
