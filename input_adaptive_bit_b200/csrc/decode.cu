@@ -24,7 +24,7 @@
 //    publishes its partial, waits until all m have arrived, and adds up its
 //    own 1/m share of the outputs over the m partials in CTA order
 //    (deterministic).
-//  * A CTA walks its range in rounds of at most 1024 units and 8 groups.  The
+//  * A CTA walks its range in rounds of at most 2048 units and 8 groups.  The
 //    segments stream through an 8-stage shared-memory ring (cp.async, 16 B per
 //    thread and copy, one barrier per 32 units).
 //  * The contraction runs on the tensor cores as m16n8k16 MMAs with fp32
@@ -53,7 +53,7 @@ constexpr int kK = 16;                // units per MMA k-step
 constexpr int kStage = 64;            // units per ring stage (4 k-steps, 2 per warp)
 constexpr int kRing = 8;              // ring stages
 constexpr int kXSlot = 6;             // first ring slot of the output CTAs' x cache
-constexpr int kRound = 1024;          // units per round
+constexpr int kRound = 2048;          // units per round
 constexpr int kSlots = 8;             // groups per window (the MMA n dimension)
 constexpr int kMaxG = kDecodeMaxDin / kGroup;
 constexpr int kXCache = 16384;        // rows of x held in shared memory

@@ -69,10 +69,11 @@ def test_optional_outputs_match_assign_bit_for_bit_or_are_skipped():
 
 def test_more_tiles_than_ctas_and_several_rounds_per_range():
     # d_out = 148 * 1024 + 16: 149 tiles (one CTA takes two), the last ragged and
-    # not 16-byte aligned (d_out / 16 odd); 10 groups and ~2500 units per tile
-    # force rounds cut both by the 8-group window and by the 1024-unit cap
+    # not 16-byte aligned (d_out / 16 odd); 10 groups with ~3.25 planes per row
+    # (~4200 units per tile) force rounds cut both by the 8-group window and by
+    # the 2048-unit cap (the first window holds ~3300 units)
     d_in, d_out = 1280, 148 * 1024 + 16
-    q, s, z, x, theta = cheap_case(2, d_in, d_out, 8)
+    q, s, z, x, theta = cheap_case(2, d_in, d_out, 8, fractions=[0.05, 0.05, 0.1, 0.2, 0.6])
     outs = np.unique(np.concatenate([np.arange(0, 64), np.arange(d_out - 80, d_out),
                                      np.random.default_rng(0).integers(0, d_out, 200)]))
     check_fused(q, s, z, x, theta, 8, outs=outs.astype(np.int32))
