@@ -533,12 +533,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
         __syncthreads();
 
         // B fragments per k-step: lane (fg, tq) holds B[2tq, 2tq+1][fg] and B[2tq+8, 2tq+9][fg];
-        // B[k][col] = x'' of unit k if the unit's group slot is col, else 0
+        // B[k][col] = x'' of unit k if the unit's group slot is col / 2 + 4 (col mod 2), else
+        // 0.  So D column 2q holds slot q and column 2q+1 slot q+4, and a window of at
+        // most 4 groups leaves the second slot of every lane empty (skipped by the flush)
         auto build_bfrag = [&]() {
           for (int q = tid; q < n_steps * 32; q += kThreads) {
             const int kk = q >> 5, L = q & 31, col = L >> 2, t2i = 2 * (L & 3);
+            const int slot_c = (col >> 1) + 4 * (col & 1);
             const uint32_t *ux = s_ux + kk * kK;
-            auto bh = [&](uint32_t e) -> uint32_t { return ((int)(e >> 16) == col) ? (e & 0xffffu) : 0u; };
+            auto bh = [&](uint32_t e) -> uint32_t { return ((int)(e >> 16) == slot_c) ? (e & 0xffffu) : 0u; };
             s_bfrag[q] = make_uint2(bh(ux[t2i]) | (bh(ux[t2i + 1]) << 16),
                                     bh(ux[t2i + 8]) | (bh(ux[t2i + 9]) << 16));
           }
@@ -626,12 +629,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
         }
         cp_async_wait<0>();
 
-        // flush: y_t += s (D 2^(24 - pos(t) + c) [+ Phi]) [+ z X] for the lane's two slots;
-        // the slice's group terms once per window (first round, even-k warps)
+        // flush: y_t += s (D 2^(24 - pos(t) + c) [+ Phi]) [+ z X] for the lane's two slots
+        // (tq and tq + 4); the slice's group terms once per window (first round, even-k warps)
         const bool terms = k0 == 0 && kp == 0;
 #pragma unroll
         for (int jj = 0; jj < 2; ++jj) {
-          const int j = 2 * tq + jj;
+          const int j = tq + 4 * jj;
           if (j < ng) {
             const SlotInfo si = s_slot[j];
             const uint16_t *srow = s_st + j * kTile + 128 * ob + 16 * fg;
