@@ -24,17 +24,18 @@
 //    publishes its partial, waits until all m have arrived, and adds up its
 //    own 1/m share of the outputs over the m partials in CTA order
 //    (deterministic).
-//  * A CTA walks its range in rounds of at most 2048 units and 8 groups.  The
-//    segments stream through an 8-stage shared-memory ring (cp.async, 16 B per
-//    thread and copy, one barrier per 32 units).
+//  * A CTA walks its range in windows of 8 groups and rounds of at most 2048
+//    units.  The segments stream through an 8-stage shared-memory ring
+//    (cp.async, 16 B per thread and copy, one barrier per 64-unit stage).
 //  * The contraction runs on the tensor cores as m16n8k16 MMAs with fp32
 //    accumulation: A (16 outputs x 16 units) is built in registers straight
 //    from the packed words -- a byte permute pairs the same 16 outputs of two
 //    units, one AND per register isolates a 2-bit field pair in the low
 //    mantissa bits of two fp16 subnormals, exactly slice * 2^(pos-24) -- and B
-//    (16 units x 8) holds x 4^(P-1-p) 2^-c_g in column (g mod 8), so the 8
-//    columns keep the 8 groups of a round apart and the group scales s are
-//    applied once per round, not per unit.  One warp covers 128 outputs with
+//    (16 units x 8) holds x 4^(P-1-p) 2^-c_g in the column of the unit's group
+//    slot j in the window (2 (j mod 4) + j / 4), so the 8 columns keep the
+//    window's 8 groups apart and the group scales s are applied once per
+//    round, not per unit.  One warp covers 128 outputs with
 //    8 MMAs per 16 units: 4 shared loads, 4 permutes, 4 shifts, 32 ANDs and
 //    8 MMAs per 512 bytes of planes, against about 240 instructions for a
 //    scalar fp32 decode of the same bytes.
