@@ -144,7 +144,7 @@ int grinqh_gemv(const uint32_t *planes, const uint16_t *s, const uint16_t *z,
  * be written by the kernel launched immediately before this call on the same
  * stream (a copy, an event or any other kernel in between lifts this).  The
  * split-K arrival wait does not give up on a correct launch; if it does (after
- * about a second) it sets the device error word to 3. */
+ * 2^20 polls, a fraction of a second) it sets the device error word to 3. */
 int grinqh_decode_gemv(const uint32_t *planes, const uint16_t *s, const uint16_t *z,
                        const uint16_t *x, const float *theta, const float *phi, int d_in,
                        int d_out, int b_max, float *y, uint8_t *b, int32_t *lists,

@@ -60,7 +60,7 @@ constexpr int kMaxG = kDecodeMaxDin / kGroup;
 constexpr int kXCache = 16384;        // rows of x held in shared memory
 constexpr int kGT = 16;               // output CTAs: threads per group, one 8-row chunk each
 constexpr int kChunkRows = 32;        // GEMV front end: rows per warp chunk, one per lane
-constexpr int kSpinLimit = 1 << 20;   // polls of a split-K counter before giving up (about 1 s)
+constexpr int kSpinLimit = 1 << 20;   // polls of a split-K counter before giving up (~0.3 s)
 constexpr int kOutCtas = 4;           // CTAs that write the optional outputs
 
 // shared memory map (bytes)

@@ -1,8 +1,9 @@
 """GPU parity of the fused decode kernel (grinqh_decode_gemv) in the cases its
 own work split creates: ranges spanning several rounds, more tiles than CTAs,
 empty groups between active ones, the largest accepted d_in, fewer units than
-CTAs, every split-K factor from 144 CTAs per tile down to one, and the
-optional outputs (bit-exact with grinqh_assign, or skipped)."""
+CTAs, every split-K factor from 144 CTAs per tile down to one, the optional
+outputs (bit-exact with grinqh_assign, or skipped), and the bounded split-K
+wait giving up with a device error instead of hanging."""
 import numpy as np
 import pytest
 import torch
@@ -139,3 +140,27 @@ def test_split_k_shares_every_ctas_per_tile(d_out):
     torch.cuda.synchronize()
     assert np.array_equal(y2.cpu().numpy().astype(np.float64), out["y"])
     grinqh_check_device_error(lin.ws)  # raises if a split-K wait gave up
+
+
+def test_split_k_wait_gives_up_and_reports_a_stale_arrival():
+    # A workspace left with one stale arrival on a tile's counter (the call
+    # requires it zeroed): the tile's last CTA to arrive waits for an arrival that
+    # never comes, gives up after its poll limit (2^20 polls), sets device
+    # error 3 and lets the kernel finish; the context stays usable.
+    from input_adaptive_bit_b200 import ERR_DEVICE, GrinqhError, grinqh_check_device_error
+    q, s, z, x, theta = cheap_case(9, 512, 1024, 8)  # one tile: every GEMV CTA shares it
+    lin = GrinqhLinear(q, s, z, 8)
+    xd, th = to_dev(x), to_dev(theta)
+    counters = lin.ws[256:260].view(torch.int32)  # the tile's arrival counter (after the header)
+    counters.fill_(1)
+    lin.decode(xd, th, outputs=False)
+    torch.cuda.synchronize()
+    with pytest.raises(GrinqhError) as err:
+        grinqh_check_device_error(lin.ws)
+    assert err.value.status == ERR_DEVICE and "code 3" in str(err.value)
+    # cleared workspace: the next call on the same layer is correct and reports nothing
+    lin.ws.zero_()
+    _, out = run_layer(None, None, None, x, theta, 8, lin=lin, path="fused")
+    b_ref = check_assign(out, x, theta, 8)
+    check_y(out, oracle.pack(q, 8), s, z, x, b_ref, 8)
+    grinqh_check_device_error(lin.ws)
