@@ -174,10 +174,10 @@ int grinqh_gemv_dense4(const uint32_t *w4, const uint16_t *s, const uint16_t *z,
  * For callers that cannot allocate device memory -- a host framework that owns
  * every byte of device memory and only hands its plug-ins streams and tensors,
  * or a latency-critical path that must never enter the allocator.  It runs
- * grinqh_assign then grinqh_gemv, keeping the assignment, lists, group sums,
- * unit stream and split-K scratch in a fixed array (about 2.7 MB) that the
- * library reserves on every GPU that loads it and holds until exit; it calls
- * no cudaMalloc/cudaFree.
+ * the fused decode kernel (grinqh_decode_gemv without its optional outputs),
+ * keeping its split-K scratch in a fixed array (about 2.2 MB) that the library
+ * reserves on every GPU that loads it and holds until exit; it calls no
+ * cudaMalloc/cudaFree.
  *   planes, s, z  the packed layer (as for grinqh_gemv); x, theta, phi as for
  *                 grinqh_assign; y fp32 [d_out] out.
  *   Limits: d_in <= 32768 and d_out <= 32768, on top of the usual shape rules;

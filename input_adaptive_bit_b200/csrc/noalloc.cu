@@ -6,11 +6,11 @@
 // memory itself and does not let plug-ins call cudaMalloc, or a latency-
 // critical path that must never reach the allocator (cudaMalloc can
 // synchronise the device).  Such a caller cannot provide the workspace that
-// grinqh_assign / grinqh_gemv need.  This entry point keeps everything that
-// is neither an input nor the output -- the precision assignment, the row
-// lists, the group sums, the unit stream, the split-K partial sums and their
-// counters -- in one fixed-size array that the library reserves on every GPU
-// that loads it and holds until the process exits.
+// grinqh_decode_gemv needs.  This entry point runs the fused decode kernel
+// (without its optional outputs) and keeps what is neither an input nor the
+// output -- the split-K partial sums, their arrival counters and the error
+// word -- in one fixed-size array that the library reserves on every GPU that
+// loads it and holds until the process exits.
 #include <mutex>
 
 #include "grinqh_internal.cuh"
@@ -22,19 +22,14 @@ constexpr int kNoAllocMaxDin = 32768;   // largest d_in this entry point accepts
 constexpr int kNoAllocMaxDout = 32768;  // largest d_out
 
 constexpr size_t a256(size_t v) { return (v + 255) & ~size_t(255); }
-// The caller-owned workspace layout (header, counters, unit stream, partial
-// sums) at the largest accepted shape, then b, lists, counts and group sums.
-constexpr size_t kWsMax =
+// The workspace layout of grinqh_workspace_bytes at the largest accepted shape
+// (header, counters, the two-call path's unit stream, partial sums).
+constexpr size_t kNoAllocBytes =
     a256(a256(a256(a256(sizeof(WsHeader) + (size_t)kMaxTiles * 4) + (size_t)kNoAllocMaxDin * 16) +
               (size_t)kNoAllocMaxDin * 16) +
          (size_t)kMaxCtas * 2 * kTileOut * 4);
-constexpr size_t kOffB = kWsMax;
-constexpr size_t kOffLists = kOffB + a256(kNoAllocMaxDin);
-constexpr size_t kOffCounts = kOffLists + a256((size_t)4 * kNoAllocMaxDin * 4);
-constexpr size_t kOffGrp = kOffCounts + 256;
-constexpr size_t kNoAllocBytes = kOffGrp + a256((size_t)2 * (kNoAllocMaxDin / kGroup) * 4);
 
-// The scratch (about 2.7 MB).  In host code this name is only a host-side
+// The scratch (about 2.2 MB).  In host code this name is only a host-side
 // stand-in; kernels get the device address from cudaGetSymbolAddress.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
 
@@ -80,18 +75,15 @@ extern "C" int grinqh_decode_gemv_noalloc(const uint32_t *planes, const uint16_t
     return record_error(GRINQH_ERR_CUDA, "grinqh_decode_gemv_noalloc: scratch address: %s",
                         cudaGetErrorString(e));
   char *sc = static_cast<char *>(base);
-  // Every call shares the array, which keeps the last call's contents; the
-  // header (device error word) and the split-K counters must start at zero.
+  // Every call shares the array, which keeps the last call's contents.  The
+  // kernel leaves its counters at zero, but the error word and the counters of a
+  // call that gave up would stay set: they are cleared first.  (The clear also
+  // keeps the kernel from overlapping the kernel before it on the stream.)
   const WsLayout L = ws_layout(d_in, d_out, b_max);
-  e = cudaMemsetAsync(sc, 0, L.unit_code, (cudaStream_t)stream);
+  e = cudaMemsetAsync(sc, 0, L.counters + (size_t)L.tiles * 4, (cudaStream_t)stream);
   if (e != cudaSuccess)
     return record_error(GRINQH_ERR_CUDA, "grinqh_decode_gemv_noalloc: clearing scratch: %s",
                         cudaGetErrorString(e));
-  float *grp = reinterpret_cast<float *>(sc + kOffGrp);
-  const int rc = grinqh_assign(x, theta, d_in, b_max, phi, reinterpret_cast<uint8_t *>(sc + kOffB),
-                               reinterpret_cast<int32_t *>(sc + kOffLists),
-                               reinterpret_cast<int32_t *>(sc + kOffCounts), grp, sc, kWsMax,
-                               stream);
-  if (rc != GRINQH_OK) return rc;
-  return grinqh_gemv(planes, s, z, grp, d_in, d_out, b_max, y, sc, kWsMax, stream);
+  return grinqh_decode_gemv(planes, s, z, x, theta, phi, d_in, d_out, b_max, y, nullptr, nullptr,
+                            nullptr, nullptr, sc, kNoAllocBytes, stream);
 }
