@@ -231,6 +231,12 @@ class Workload:
         self.graphs = []
         self.gemv_graph = None
         self.two_graph = None
+        self.groups = self.layer_groups()
+        self.group_graph = self.single_graph = None
+        if self.groups is not None:
+            from input_adaptive_bit_b200 import grinqh_group_workspace_bytes
+            self.group_ws = torch.zeros(grinqh_group_workspace_bytes(), dtype=torch.uint8,
+                                        device=device)
 
     def xv(self, k, j):
         return self.x_dev[k, self.offsets[j]:self.offsets[j + 1]]
@@ -238,11 +244,43 @@ class Workload:
     def yv(self, j):
         return self.y_dev[self.y_offsets[j]:self.y_offsets[j + 1]]
 
-    def launch_step(self, k, stream, path=None):
+    def layer_groups(self):
+        """The layer-stack workload's linears in launch order, the independent ones of a
+        layer (q, k, v; gate, up) in one group each; None for the other workloads."""
+        if not all("." in s.name for s in self.specs):
+            return None
+        groups, key_prev = [], None
+        for j, spec in enumerate(self.specs):
+            layer, kind = spec.name.split(".", 1)
+            key = (layer, {"q": "qkv", "k": "qkv", "v": "qkv", "gate": "gu", "up": "gu"}.get(kind, kind))
+            if key == key_prev:
+                groups[-1].append(j)
+            else:
+                groups.append([j])
+            key_prev = key
+        return groups
+
+    def launch_step_grouped(self, k, stream):
+        """One step with each group of independent linears in one grouped launch (no
+        optional outputs)."""
+        from input_adaptive_bit_b200 import grinqh_decode_gemv_group
+        for grp in self.groups:
+            if len(grp) == 1:
+                j = grp[0]
+                self.layers[j].decode(self.xv(k, j), self.thetas[j], y=self.yv(j), outputs=False,
+                                      stream=stream)
+                continue
+            lins = [(self.layers[j].planes, self.layers[j].s, self.layers[j].z, self.xv(k, j),
+                     self.thetas[j], None, self.layers[j].d_in, self.layers[j].d_out,
+                     self.layers[j].b_max, self.yv(j)) for j in grp]
+            grinqh_decode_gemv_group(lins, self.group_ws, self.group_ws.numel(), stream=stream)
+
+    def launch_step(self, k, stream, path=None, outputs=True):
         path = path or self.path
         for j, lin in enumerate(self.layers):
             if path == "fused":
-                lin.decode(self.xv(k, j), self.thetas[j], y=self.yv(j), stream=stream)
+                lin.decode(self.xv(k, j), self.thetas[j], y=self.yv(j), outputs=outputs,
+                           stream=stream)
             else:
                 lin.assign(self.xv(k, j), self.thetas[j], stream=stream)
                 lin.gemv(self.yv(j), stream=stream)
@@ -272,6 +310,18 @@ class Workload:
         with torch.cuda.graph(g, stream=self.stream):
             self.launch_gemvs(self.stream)
         self.gemv_graph = g
+        if self.groups is not None:  # layer stack: grouped launches, and the same without outputs
+            with torch.cuda.stream(self.stream):
+                self.launch_step_grouped(0, self.stream)
+                self.launch_step(0, self.stream, outputs=False)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=self.stream):
+                self.launch_step_grouped(0, self.stream)
+            self.group_graph = g
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=self.stream):
+                self.launch_step(0, self.stream, outputs=False)
+            self.single_graph = g
         torch.cuda.synchronize(self.device)
 
     def bytes_per_pool_entry(self, include_x=True):
@@ -592,6 +642,19 @@ def main(argv=None):
         launch_us = gemv_launch_us
         bytes_launch = gemv_bytes[0] / n_gemv
     achieved = bytes_launch / (launch_us * 1e-6) / 1e9
+    grouped = None
+    if wl.group_graph is not None:
+        with torch.cuda.stream(wl.stream):
+            ms_grp = device_time_ms(torch, wl.stream, lambda i: wl.group_graph.replay(), reps)
+            ms_one = device_time_ms(torch, wl.stream, lambda i: wl.single_graph.replay(), reps)
+        ms_grp = max_over_ranks(dist, ms_grp, device)
+        ms_one = max_over_ranks(dist, ms_one, device)
+        grouped = {"launches_per_step": len(wl.groups),
+                   "ms_per_step": round(ms_grp / reps, 5),
+                   "value": round(step_bytes[0] / (ms_grp / reps * 1e-3) / 1e9, 1),
+                   "ungrouped_no_outputs_ms_per_step": round(ms_one / reps, 5),
+                   "how": "q/k/v and gate/up of each layer in one grinqh_decode_gemv_group launch; "
+                          "no optional outputs in either graph; pool entry 0"}
     two_kernel = {"ms_per_step": round(ms_two / reps, 5),
                   "value": round(step_bytes[0] / (ms_two / reps * 1e-3) / 1e9, 1),
                   "gemv_us_per_launch": round(gemv_launch_us, 3),
@@ -667,6 +730,7 @@ def main(argv=None):
         "gpu_launches": (1 if args.path == "fused" else 2) * n_gemv * args.steps,
         "path": args.path,
         "two_kernel_path": two_kernel,
+        **({"grouped_layers": grouped} if grouped is not None else {}),
         "clocks": clocks,
         "cpu_baseline": cpu,
     }

@@ -151,6 +151,38 @@ int grinqh_decode_gemv(const uint32_t *planes, const uint16_t *s, const uint16_t
                        int32_t *counts, float *grp_sums, void *ws, size_t ws_bytes,
                        void *stream);
 
+/* ---- Grouped decode (several independent linears in one launch) -------------
+ * The linears of a decoder layer that do not depend on each other -- q, k and
+ * v, or gate and up -- each run as grinqh_decode_gemv would (every linear its
+ * own x, theta, phi and y), but in one kernel launch: the GPU's CTAs are split
+ * between them in proportion to their plane bytes, so the launch's fixed costs
+ * (the wait on the kernel before, the per-CTA front end, the split-K tail) are
+ * paid once for the group.  The optional outputs (b, lists, counts, group sums)
+ * are not produced.  Each linear obeys the rules of grinqh_decode_gemv (d_in
+ * <= 65536, alignment, theta and phi not written by the kernel launched just
+ * before).  y of a linear equals its single-call y within the summation-order
+ * rounding (its CTAs take different row slices).
+ *   n      1 .. GRINQH_MAX_GROUP linears.
+ *   lins   host array of n descriptors (read during the call only).
+ *   ws     workspace of grinqh_group_workspace_bytes() bytes (zero-filled once;
+ *          left zeroed), not shared with a concurrent call. */
+#define GRINQH_MAX_GROUP 4
+typedef struct grinqh_linear {
+  const uint32_t *planes; /* as for grinqh_decode_gemv */
+  const uint16_t *s;
+  const uint16_t *z;
+  const uint16_t *x;
+  const float *theta;
+  const float *phi; /* NULL: the default table */
+  int d_in;
+  int d_out;
+  int b_max;
+  float *y; /* fp32 [d_out] out */
+} grinqh_linear;
+size_t grinqh_group_workspace_bytes(void);
+int grinqh_decode_gemv_group(int n, const grinqh_linear *lins, void *ws, size_t ws_bytes,
+                             void *stream);
+
 /* Reads and clears the device error word of `ws` (synchronises `stream`).
  * Returns GRINQH_OK, or GRINQH_ERR_DEVICE with the device code in
  * grinqh_last_error(). */

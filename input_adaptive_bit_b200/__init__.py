@@ -18,7 +18,9 @@ __all__ = [
     "GrinqhError", "lib", "lib_path", "grinqh_version", "grinqh_last_error",
     "grinqh_workspace_bytes", "grinqh_pack", "grinqh_unpack", "grinqh_assign", "grinqh_gemv",
     "grinqh_check_device_error", "grinqh_pack_dense4", "grinqh_dense4_workspace_bytes",
-    "grinqh_gemv_dense4", "grinqh_decode_gemv", "grinqh_decode_gemv_noalloc", "EXPORTS",
+    "grinqh_gemv_dense4", "grinqh_decode_gemv", "grinqh_decode_gemv_noalloc",
+    "grinqh_group_workspace_bytes", "grinqh_decode_gemv_group", "GrinqhLinearDesc", "MAX_GROUP",
+    "EXPORTS",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -30,6 +32,17 @@ ERR_UNSUPPORTED_SHAPE = -2
 ERR_WORKSPACE_TOO_SMALL = -3
 ERR_CUDA = -4
 ERR_DEVICE = -5
+
+MAX_GROUP = 4  # GRINQH_MAX_GROUP
+
+
+class GrinqhLinearDesc(ctypes.Structure):
+    """struct grinqh_linear: one linear of a grouped decode call (include/grinqh.h)."""
+    _fields_ = [("planes", ctypes.c_void_p), ("s", ctypes.c_void_p), ("z", ctypes.c_void_p),
+                ("x", ctypes.c_void_p), ("theta", ctypes.c_void_p), ("phi", ctypes.c_void_p),
+                ("d_in", ctypes.c_int), ("d_out", ctypes.c_int), ("b_max", ctypes.c_int),
+                ("y", ctypes.c_void_p)]
+
 
 # name -> (restype, argtypes); p = pointer (passed as c_void_p), i = int, z = size_t
 _P, _I, _Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
@@ -48,6 +61,8 @@ EXPORTS = {
     "grinqh_decode_gemv": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _P, _P, _P, _P, _P, _P,
                                 _Z, _P]),
     "grinqh_decode_gemv_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _P, _P]),
+    "grinqh_group_workspace_bytes": (_Z, []),
+    "grinqh_decode_gemv_group": (_I, [_I, _P, _P, _Z, _P]),
 }
 
 
@@ -158,8 +173,23 @@ def grinqh_decode_gemv(planes, s, z, x, theta, phi, d_in, d_out, b_max, y, b, li
 
 
 def grinqh_decode_gemv_noalloc(planes, s, z, x, theta, phi, d_in, d_out, b_max, y, stream=None):
-    """assign + gemv with the library's fixed scratch: for callers that cannot
-    allocate device memory (see include/grinqh.h for limits and sharing)."""
+    """The fused decode kernel on the library's fixed scratch: for callers that
+    cannot allocate device memory (see include/grinqh.h for limits and sharing)."""
     _check(lib().grinqh_decode_gemv_noalloc(_ptr(planes), _ptr(s), _ptr(z), _ptr(x), _ptr(theta),
                                             _ptr(phi), d_in, d_out, b_max, _ptr(y),
                                             _stream(stream)))
+
+
+def grinqh_group_workspace_bytes() -> int:
+    return lib().grinqh_group_workspace_bytes()
+
+
+def grinqh_decode_gemv_group(lins, ws, ws_bytes, stream=None):
+    """Several independent linears in one launch.  `lins` is a sequence of
+    (planes, s, z, x, theta, phi, d_in, d_out, b_max, y) tuples (phi may be None)."""
+    arr = (GrinqhLinearDesc * max(1, len(lins)))()
+    for j, (planes, s, z, x, theta, phi, d_in, d_out, b_max, y) in enumerate(lins):
+        arr[j] = GrinqhLinearDesc(_ptr(planes), _ptr(s), _ptr(z), _ptr(x), _ptr(theta), _ptr(phi),
+                                  d_in, d_out, b_max, _ptr(y))
+    _check(lib().grinqh_decode_gemv_group(len(lins), ctypes.cast(arr, ctypes.c_void_p), _ptr(ws),
+                                          ws_bytes, _stream(stream)))

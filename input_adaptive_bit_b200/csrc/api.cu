@@ -210,6 +210,44 @@ int grinqh_decode_gemv(const uint32_t *planes, const uint16_t *s, const uint16_t
                      "grinqh_decode_gemv launch");
 }
 
+size_t grinqh_group_workspace_bytes(void) { return grinqh::group_ws_bytes(); }
+
+int grinqh_decode_gemv_group(int n, const grinqh_linear *lins, void *ws, size_t ws_bytes,
+                             void *stream) {
+  if (n < 1 || n > GRINQH_MAX_GROUP)
+    return fail(GRINQH_ERR_INVALID_ARG, "grinqh_decode_gemv_group: n must be in [1, %d] (got %d)",
+                GRINQH_MAX_GROUP, n);
+  TRY(check_ptr(lins, alignof(grinqh_linear), "lins"));
+  long long tiles = 0;
+  for (int j = 0; j < n; ++j) {
+    const grinqh_linear &l = lins[j];
+    TRY(check_bmax(l.b_max));
+    TRY(check_din(l.d_in));
+    TRY(check_dout(l.d_out));
+    if (l.d_in > grinqh::kDecodeMaxDin)
+      return fail(GRINQH_ERR_UNSUPPORTED_SHAPE,
+                  "grinqh_decode_gemv_group: linear %d: d_in must be <= %d (got %d)", j,
+                  grinqh::kDecodeMaxDin, l.d_in);
+    TRY(check_ptr(l.planes, (l.d_out / 16) % 4 == 0 ? 16 : 4, "planes"));
+    TRY(check_ptr(l.s, 16, "s"));
+    TRY(check_ptr(l.z, 16, "z"));
+    TRY(check_ptr(l.x, 16, "x"));
+    TRY(check_ptr(l.theta, 4, "theta"));
+    if (l.phi) TRY(check_ptr(l.phi, 4, "phi"));
+    TRY(check_ptr(l.y, 4, "y"));
+    tiles += (l.d_out + 1023) / 1024;
+  }
+  if (tiles > grinqh::kMaxTiles)
+    return fail(GRINQH_ERR_UNSUPPORTED_SHAPE, "grinqh_decode_gemv_group: too many output tiles (%lld)",
+                tiles);
+  TRY(check_ptr(ws, 256, "ws"));
+  if (ws_bytes < grinqh::group_ws_bytes())
+    return fail(GRINQH_ERR_WORKSPACE_TOO_SMALL, "workspace of %zu bytes, a group needs %zu",
+                ws_bytes, grinqh::group_ws_bytes());
+  return cuda_status(grinqh::launch_decode_group(n, lins, ws, (cudaStream_t)stream),
+                     "grinqh_decode_gemv_group launch");
+}
+
 int grinqh_check_device_error(void *ws, void *stream) {
   TRY(check_ptr(ws, 256, "ws"));
   int code = 0;

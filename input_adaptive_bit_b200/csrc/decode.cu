@@ -62,6 +62,12 @@ constexpr int kGT = 16;               // output CTAs: threads per group, one 8-r
 constexpr int kChunkRows = 32;        // GEMV front end: rows per warp chunk, one per lane
 constexpr int kSpinLimit = 1 << 20;   // polls of a split-K counter before giving up (~0.3 s)
 constexpr int kOutCtas = 4;           // CTAs that write the optional outputs
+constexpr int kMaxGroup = GRINQH_MAX_GROUP;  // linears of one grouped launch
+
+// workspace of a grouped launch: the header, the arrival counters of every
+// linear's tiles (fixed offset), then the partial tiles of every CTA
+constexpr size_t kGroupWsCounters = sizeof(WsHeader);
+constexpr size_t kGroupWsPartials = (kGroupWsCounters + (size_t)kMaxTiles * 4 + 255) & ~size_t(255);
 
 // shared memory map (bytes)
 constexpr size_t kStageBytes = (size_t)kStage * kRow * 4;
@@ -119,8 +125,17 @@ struct DecodeArgs {
   int32_t *counts;
   float *grp_sums;
   unsigned *counters;
-  float *partials;    // [gridDim.x][kTile]
+  float *partials;    // [CTAs of this linear][kTile]
   int *error;         // the workspace's device error word
+  int reserve_out;    // set aside the output CTAs (the single call does, whether or not
+                      // outputs are asked for, so y never depends on it; a group does not)
+};
+
+// The linears of one launch: CTAs [cta_start[j], cta_start[j+1]) run linear j.
+struct DecodeGroup {
+  int n;
+  int cta_start[kMaxGroup + 1];
+  DecodeArgs lin[kMaxGroup];
 };
 
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
@@ -296,7 +311,7 @@ __device__ __forceinline__ void write_outputs(const DecodeArgs &a, unsigned char
 }
 
 template <bool ALIGNED>
-__global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
+__global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_constant__ DecodeGroup g) {
   extern __shared__ __align__(128) unsigned char smem[];
   uint32_t *ring = reinterpret_cast<uint32_t *>(smem + kSmRing);
   int32_t *s_region = reinterpret_cast<int32_t *>(smem + kSmRegion);
@@ -311,14 +326,19 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
   const int fg = lane >> 2, tq = lane & 3;  // MMA fragment row group and column pair
   const int ob = warp & (kBlocks - 1);      // the warp's 128-output block of the tile
   const int kp = warp / kBlocks;            // ... and its k-step parity
-  const int C = gridDim.x, c = blockIdx.x;
+  // this CTA's linear, and the CTAs that linear has
+  int jl = 0;
+#pragma unroll
+  for (int i = 1; i < kMaxGroup; ++i) jl += (i < g.n && (int)blockIdx.x >= g.cta_start[i]) ? 1 : 0;
+  const DecodeArgs &a = g.lin[jl];
+  const int C = g.cta_start[jl + 1] - g.cta_start[jl], c = (int)blockIdx.x - g.cta_start[jl];
   const int P = a.P;
 
   // ---- what depends on the shapes only: computed before the wait below, so it
   // overlaps the tail of the kernel launched before (programmatic launch) ----
   // the last CTAs write the optional outputs, the others run the GEMV; they are
   // set aside whether or not outputs are asked for, so y does not depend on it
-  const int n_out = C > 2 * kOutCtas ? kOutCtas : 1;
+  const int n_out = !a.reserve_out ? 0 : (C > 2 * kOutCtas ? kOutCtas : 1);
   const int C_g = C - n_out;
   // tiles x row slices: m CTAs per tile, CTA `part` takes the 8-row chunks
   // [R8 part / m, R8 (part + 1) / m); more tiles than CTAs: whole tiles in turn
@@ -783,11 +803,11 @@ int device_sms() {
 }
 
 template <bool ALIGNED>
-cudaError_t launch_variant(const DecodeArgs &a, cudaStream_t st) {
+cudaError_t launch_variant(const DecodeGroup &g, cudaStream_t st) {
   cudaError_t e = ensure_smem_attr((const void *)decode_kernel<ALIGNED>, kSmBytes);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(device_sms());
+  cfg.gridDim = dim3(g.cta_start[g.n]);
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = kSmBytes;
   cfg.stream = st;
@@ -796,18 +816,13 @@ cudaError_t launch_variant(const DecodeArgs &a, cudaStream_t st) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, decode_kernel<ALIGNED>, a);
+  return cudaLaunchKernelEx(&cfg, decode_kernel<ALIGNED>, g);
 }
 
-}  // namespace
-
-cudaError_t launch_decode(const uint32_t *planes, const uint16_t *s, const uint16_t *z,
-                          const uint16_t *x, const float *theta, const float *phi, int d_in,
-                          int d_out, int b_max, float *y, uint8_t *b, int32_t *lists,
-                          int32_t *counts, float *grp_sums, void *ws, cudaStream_t st) {
-  const WsLayout L = ws_layout(d_in, d_out, b_max);
-  char *w = static_cast<char *>(ws);
-  DecodeArgs a;
+DecodeArgs make_args(const uint32_t *planes, const uint16_t *s, const uint16_t *z,
+                     const uint16_t *x, const float *theta, const float *phi, int d_in, int d_out,
+                     int b_max, float *y) {
+  DecodeArgs a = {};
   a.planes = planes;
   a.s = s;
   a.z = z;
@@ -822,6 +837,31 @@ cudaError_t launch_decode(const uint32_t *planes, const uint16_t *s, const uint1
   a.G = d_in / kGroup;
   a.tiles = (d_out + kTile - 1) / kTile;
   a.y = y;
+  return a;
+}
+
+cudaError_t launch_group(DecodeGroup &g, cudaStream_t st) {
+  bool aligned = true;  // 16-byte plane copies need every linear's rows 16-byte aligned
+  for (int j = 0; j < g.n; ++j) aligned = aligned && g.lin[j].W % 4 == 0;
+  cudaError_t e = aligned ? launch_variant<true>(g, st) : launch_variant<false>(g, st);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_decode(const uint32_t *planes, const uint16_t *s, const uint16_t *z,
+                          const uint16_t *x, const float *theta, const float *phi, int d_in,
+                          int d_out, int b_max, float *y, uint8_t *b, int32_t *lists,
+                          int32_t *counts, float *grp_sums, void *ws, cudaStream_t st) {
+  const WsLayout L = ws_layout(d_in, d_out, b_max);
+  char *w = static_cast<char *>(ws);
+  DecodeGroup g = {};
+  g.n = 1;
+  g.cta_start[0] = 0;
+  g.cta_start[1] = device_sms();
+  DecodeArgs &a = g.lin[0];
+  a = make_args(planes, s, z, x, theta, phi, d_in, d_out, b_max, y);
   a.b = b;
   a.lists = lists;
   a.counts = counts;
@@ -829,9 +869,50 @@ cudaError_t launch_decode(const uint32_t *planes, const uint16_t *s, const uint1
   a.counters = reinterpret_cast<unsigned *>(w + L.counters);
   a.partials = reinterpret_cast<float *>(w + L.partials);
   a.error = &reinterpret_cast<WsHeader *>(w)->error;
-  cudaError_t e = (a.W % 4 == 0) ? launch_variant<true>(a, st) : launch_variant<false>(a, st);
-  if (e != cudaSuccess) return e;
-  return cudaGetLastError();
+  a.reserve_out = 1;
+  return launch_group(g, st);
+}
+
+size_t group_ws_bytes() { return kGroupWsPartials + (size_t)kMaxCtas * kTile * 4; }
+
+cudaError_t launch_decode_group(int n, const grinqh_linear *lins, void *ws, cudaStream_t st) {
+  char *w = static_cast<char *>(ws);
+  DecodeGroup g = {};
+  g.n = n;
+  // CTAs in proportion to each linear's plane bytes (tiles x d_in x P), at least one each
+  const int C = device_sms();
+  double tot = 0.0, wgt[kMaxGroup];
+  for (int j = 0; j < n; ++j) {
+    const int tiles = (lins[j].d_out + kTile - 1) / kTile;
+    wgt[j] = (double)tiles * lins[j].d_in * (lins[j].b_max / 2);
+    tot += wgt[j];
+  }
+  int cnt[kMaxGroup], used = 0;
+  for (int j = 0; j < n; ++j) {
+    cnt[j] = (int)((double)C * wgt[j] / tot);
+    if (cnt[j] < 1) cnt[j] = 1;
+    used += cnt[j];
+  }
+  while (used > C) {  // rounding up the small ones may overshoot: trim the largest
+    int big = 0;
+    for (int j = 1; j < n; ++j)
+      if (cnt[j] > cnt[big]) big = j;
+    --cnt[big];
+    --used;
+  }
+  int tile_off = 0;
+  for (int j = 0; j < n; ++j) {
+    const grinqh_linear &l = lins[j];
+    g.cta_start[j + 1] = g.cta_start[j] + cnt[j];
+    DecodeArgs &a = g.lin[j];
+    a = make_args(l.planes, l.s, l.z, l.x, l.theta, l.phi, l.d_in, l.d_out, l.b_max, l.y);
+    a.counters = reinterpret_cast<unsigned *>(w + kGroupWsCounters) + tile_off;
+    a.partials = reinterpret_cast<float *>(w + kGroupWsPartials) + (size_t)g.cta_start[j] * kTile;
+    a.error = &reinterpret_cast<WsHeader *>(w)->error;
+    a.reserve_out = 0;
+    tile_off += a.tiles;
+  }
+  return launch_group(g, st);
 }
 
 }  // namespace grinqh

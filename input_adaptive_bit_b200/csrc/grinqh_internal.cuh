@@ -189,6 +189,8 @@ cudaError_t launch_decode(const uint32_t *planes, const uint16_t *s, const uint1
                           const uint16_t *x, const float *theta, const float *phi, int d_in,
                           int d_out, int b_max, float *y, uint8_t *b, int32_t *lists,
                           int32_t *counts, float *grp_sums, void *ws, cudaStream_t st);
+cudaError_t launch_decode_group(int n, const grinqh_linear *lins, void *ws, cudaStream_t st);
+size_t group_ws_bytes();
 cudaError_t launch_pack_dense4(const uint8_t *q4, int d_in, int d_out, uint32_t *w4,
                                cudaStream_t st);
 size_t dense4_ws_bytes(int d_in, int d_out);

@@ -124,6 +124,29 @@ def test_decode_argument_checks():
     assert _status("grinqh_decode_gemv", *unaligned_x) == gq.ERR_INVALID_ARG
 
 
+def test_group_argument_checks():
+    need = gq.grinqh_group_workspace_bytes()
+    assert need >= 256 + 128 * 1024
+    lin = gq.GrinqhLinearDesc(FAKE, FAKE, FAKE, FAKE, FAKE, None, 256, 64, 8, FAKE)
+    arr = (gq.GrinqhLinearDesc * 5)(*([lin] * 5))
+    p = ctypes.cast(arr, ctypes.c_void_p)
+    lib = gq.lib()
+    assert lib.grinqh_decode_gemv_group(0, p, FAKE, need, None) == gq.ERR_INVALID_ARG
+    assert lib.grinqh_decode_gemv_group(gq.MAX_GROUP + 1, p, FAKE, need, None) == gq.ERR_INVALID_ARG
+    assert lib.grinqh_decode_gemv_group(2, None, FAKE, need, None) == gq.ERR_INVALID_ARG
+    assert lib.grinqh_decode_gemv_group(2, p, FAKE, need - 1, None) == gq.ERR_WORKSPACE_TOO_SMALL
+    assert lib.grinqh_decode_gemv_group(2, p, None, need, None) == gq.ERR_INVALID_ARG
+    arr[1].y = None
+    assert lib.grinqh_decode_gemv_group(2, p, FAKE, need, None) == gq.ERR_INVALID_ARG
+    arr[1].y = FAKE
+    arr[1].d_in = 65536 + 128
+    assert lib.grinqh_decode_gemv_group(2, p, FAKE, need, None) == gq.ERR_UNSUPPORTED_SHAPE
+    assert "65536" in gq.grinqh_last_error()
+    arr[1].d_in = 256
+    arr[1].b_max = 5
+    assert lib.grinqh_decode_gemv_group(2, p, FAKE, need, None) == gq.ERR_INVALID_ARG
+
+
 def test_dense4_argument_checks():
     need = gq.grinqh_dense4_workspace_bytes(256, 64)
     assert need > 0

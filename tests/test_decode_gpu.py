@@ -164,3 +164,32 @@ def test_split_k_wait_gives_up_and_reports_a_stale_arrival():
     b_ref = check_assign(out, x, theta, 8)
     check_y(out, oracle.pack(q, 8), s, z, x, b_ref, 8)
     grinqh_check_device_error(lin.ws)
+
+
+@pytest.mark.parametrize("shapes", [
+    [(2048, 2048, 8), (2048, 512, 8), (2048, 512, 8)],            # q, k, v of one layer
+    [(1024, 4096, 8), (4096, 1024, 8)],                           # different d_in
+    [(512, 1040, 6), (1024, 3072, 4), (256, 16, 2), (2048, 1024, 8)],  # mixed widths, a ragged unaligned layout
+    [(1024, 2048, 8)],                                            # a group of one
+])
+def test_grouped_launch_matches_the_oracle_per_linear(shapes):
+    from input_adaptive_bit_b200 import (grinqh_check_device_error, grinqh_decode_gemv_group,
+                                         grinqh_group_workspace_bytes)
+    cases, lins = [], []
+    for i, (d_in, d_out, b_max) in enumerate(shapes):
+        q, s, z, x, theta = cheap_case(20 + i, d_in, d_out, b_max)
+        lin = GrinqhLinear(q, s, z, b_max)
+        xd, th = to_dev(x), to_dev(theta)
+        y = torch.full((d_out,), float("nan"), dtype=torch.float32, device="cuda")
+        cases.append((q, s, z, x, theta, b_max, lin, xd, th, y))
+    nbytes = grinqh_group_workspace_bytes()
+    ws = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
+    for _ in range(2):  # twice: the counters must come back to zero
+        grinqh_decode_gemv_group([(c[6].planes, c[6].s, c[6].z, c[7], c[8], None, c[6].d_in,
+                                   c[6].d_out, c[5], c[9]) for c in cases], ws, nbytes)
+        torch.cuda.synchronize()
+        for q, s, z, x, theta, b_max, lin, xd, th, y in cases:
+            out = {"y": y.cpu().numpy().astype(np.float64)}
+            check_y(out, oracle.pack(q, b_max), s, z, x, oracle.assign(x, theta, b_max), b_max)
+    grinqh_check_device_error(ws)
+    assert not ws[256:256 + 4 * 64].any()  # every arrival counter is back at zero
