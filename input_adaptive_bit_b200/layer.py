@@ -9,7 +9,8 @@ from __future__ import annotations
 
 import torch
 
-from . import (grinqh_assign, grinqh_decode_gemv, grinqh_gemv, grinqh_gemv_dense4, grinqh_pack,
+from . import (MAX_GROUP, grinqh_decode_gemv_group, grinqh_group_workspace_bytes,
+               grinqh_assign, grinqh_decode_gemv, grinqh_gemv, grinqh_gemv_dense4, grinqh_pack,
                grinqh_pack_dense4, grinqh_dense4_workspace_bytes, grinqh_workspace_bytes)
 
 GROUP = 128
@@ -75,6 +76,28 @@ class GrinqhLinear:
         """x: fp16 [d_in] on the device; theta: fp32 [b_max/2] on the device."""
         self.assign(x, theta, phi, stream)
         return self.gemv(y, stream)
+
+
+class DecodeGroup:
+    """Independent GrinqhLinear layers (q, k, v of a decoder layer; gate, up) decoded in
+    one launch of grinqh_decode_gemv_group; holds the group's workspace."""
+
+    def __init__(self, layers, device="cuda"):
+        if not 1 <= len(layers) <= MAX_GROUP:
+            raise ValueError(f"a group holds 1..{MAX_GROUP} layers, got {len(layers)}")
+        self.layers = list(layers)
+        self.ws_bytes = grinqh_group_workspace_bytes()
+        self.ws = torch.zeros(self.ws_bytes, dtype=torch.uint8, device=torch.device(device))
+
+    def __call__(self, xs, thetas, phis=None, ys=None, stream=None):
+        """xs, thetas (and phis, ys if given): one per layer; returns the ys."""
+        phis = phis or [None] * len(self.layers)
+        ys = ys or [lin.y for lin in self.layers]
+        grinqh_decode_gemv_group(
+            [(lin.planes, lin.s, lin.z, x, th, ph, lin.d_in, lin.d_out, lin.b_max, y)
+             for lin, x, th, ph, y in zip(self.layers, xs, thetas, phis, ys)],
+            self.ws, self.ws_bytes, stream)
+        return ys
 
 
 class Dense4Linear:

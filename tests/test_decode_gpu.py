@@ -193,3 +193,14 @@ def test_grouped_launch_matches_the_oracle_per_linear(shapes):
             check_y(out, oracle.pack(q, b_max), s, z, x, oracle.assign(x, theta, b_max), b_max)
     grinqh_check_device_error(ws)
     assert not ws[256:256 + 4 * 64].any()  # every arrival counter is back at zero
+
+
+def test_decode_group_helper_of_the_layer_module():
+    from input_adaptive_bit_b200.layer import DecodeGroup
+    cases = [cheap_case(30 + i, d_in, d_out, 8) for i, (d_in, d_out) in enumerate([(1024, 2048), (1024, 512)])]
+    layers = [GrinqhLinear(q, s, z, 8) for q, s, z, _, _ in cases]
+    ys = DecodeGroup(layers)([to_dev(c[3]) for c in cases], [to_dev(c[4]) for c in cases])
+    torch.cuda.synchronize()
+    for (q, s, z, x, theta), y in zip(cases, ys):
+        out = {"y": y.cpu().numpy().astype(np.float64)}
+        check_y(out, oracle.pack(q, 8), s, z, x, oracle.assign(x, theta, 8), 8)
