@@ -78,7 +78,7 @@ int record_error(int code, const char *fmt, ...) {
 cudaError_t ensure_smem_attr(const void *kernel, size_t bytes) {
   // One bit per (device, kernel slot); a handful of kernels use this.
   static std::atomic<unsigned long long> done[64];
-  static const void *slots[8];
+  static const void *slots[16];
   static std::atomic<int> n_slots{0};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -88,7 +88,7 @@ cudaError_t ensure_smem_attr(const void *kernel, size_t bytes) {
     if (slots[i] == kernel) slot = i;
   if (slot < 0) {
     slot = n_slots.fetch_add(1);
-    if (slot >= 8) return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (slot >= 16) return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
     slots[slot] = kernel;
   }
   const unsigned long long bit = 1ull << slot;

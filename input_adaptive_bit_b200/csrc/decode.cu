@@ -310,7 +310,7 @@ __device__ __forceinline__ void write_outputs(const DecodeArgs &a, unsigned char
   }
 }
 
-template <bool ALIGNED>
+template <bool ALIGNED, bool GROUPED>
 __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_constant__ DecodeGroup g) {
   extern __shared__ __align__(128) unsigned char smem[];
   uint32_t *ring = reinterpret_cast<uint32_t *>(smem + kSmRing);
@@ -326,10 +326,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
   const int fg = lane >> 2, tq = lane & 3;  // MMA fragment row group and column pair
   const int ob = warp & (kBlocks - 1);      // the warp's 128-output block of the tile
   const int kp = warp / kBlocks;            // ... and its k-step parity
-  // this CTA's linear, and the CTAs that linear has
+  // this CTA's linear, and the CTAs that linear has (a single linear: a fixed index,
+  // so its arguments are read at fixed offsets)
   int jl = 0;
+  if (GROUPED) {
 #pragma unroll
-  for (int i = 1; i < kMaxGroup; ++i) jl += (i < g.n && (int)blockIdx.x >= g.cta_start[i]) ? 1 : 0;
+    for (int i = 1; i < kMaxGroup; ++i) jl += (i < g.n && (int)blockIdx.x >= g.cta_start[i]) ? 1 : 0;
+  }
   const DecodeArgs &a = g.lin[jl];
   const int C = g.cta_start[jl + 1] - g.cta_start[jl], c = (int)blockIdx.x - g.cta_start[jl];
   const int P = a.P;
@@ -802,9 +805,9 @@ int device_sms() {
   return n;
 }
 
-template <bool ALIGNED>
+template <bool ALIGNED, bool GROUPED>
 cudaError_t launch_variant(const DecodeGroup &g, cudaStream_t st) {
-  cudaError_t e = ensure_smem_attr((const void *)decode_kernel<ALIGNED>, kSmBytes);
+  cudaError_t e = ensure_smem_attr((const void *)decode_kernel<ALIGNED, GROUPED>, kSmBytes);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(g.cta_start[g.n]);
@@ -816,7 +819,7 @@ cudaError_t launch_variant(const DecodeGroup &g, cudaStream_t st) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, decode_kernel<ALIGNED>, g);
+  return cudaLaunchKernelEx(&cfg, decode_kernel<ALIGNED, GROUPED>, g);
 }
 
 DecodeArgs make_args(const uint32_t *planes, const uint16_t *s, const uint16_t *z,
@@ -843,7 +846,11 @@ DecodeArgs make_args(const uint32_t *planes, const uint16_t *s, const uint16_t *
 cudaError_t launch_group(DecodeGroup &g, cudaStream_t st) {
   bool aligned = true;  // 16-byte plane copies need every linear's rows 16-byte aligned
   for (int j = 0; j < g.n; ++j) aligned = aligned && g.lin[j].W % 4 == 0;
-  cudaError_t e = aligned ? launch_variant<true>(g, st) : launch_variant<false>(g, st);
+  cudaError_t e;
+  if (g.n == 1)
+    e = aligned ? launch_variant<true, false>(g, st) : launch_variant<false, false>(g, st);
+  else
+    e = aligned ? launch_variant<true, true>(g, st) : launch_variant<false, true>(g, st);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
