@@ -55,7 +55,7 @@ NCU_TRAFFIC = {
     # gemv.cu, grinqh_gemv (profiles/grinqh_gemv_qwen3-8b-proj_launches.md)
     "84585736bc0dc9cf2ac9f0a4738586346a63ac0a4e44acbdc753bb3917df6db4": 17150844,
     # decode.cu, grinqh_decode_gemv (profiles/decode_kernel_qwen3-8b-proj_launches.md)
-    "5487a95c442720bebdbe6680fc7f247e32972d89fb40413bac6c252b4bd007b6": 17112529,
+    "3b99529ba0960d7a26a4dd1bbdabdf74e36c38bd2fd67450277be62133263a3e": 17112247,
 }
 KERNEL_SOURCE = {"fused": "decode.cu", "two": "gemv.cu"}
 
