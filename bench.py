@@ -245,20 +245,25 @@ class Workload:
         return self.y_dev[self.y_offsets[j]:self.y_offsets[j + 1]]
 
     def layer_groups(self):
-        """The layer-stack workload's linears in launch order, the independent ones of a
-        layer (q, k, v; gate, up) in one group each; None for the other workloads."""
-        if not all("." in s.name for s in self.specs):
-            return None
+        """The linears in launch order with the independent ones of a layer (q, k, v;
+        gate, up) in one group each -- names "L<layer>.<kind>" or "<kind>_proj@<bits>";
+        None when no two linears group."""
         groups, key_prev = [], None
         for j, spec in enumerate(self.specs):
-            layer, kind = spec.name.split(".", 1)
+            if "." in spec.name:
+                layer, kind = spec.name.split(".", 1)
+            elif "@" in spec.name:
+                kind, layer = spec.name.split("@", 1)
+            else:
+                return None
+            kind = kind.replace("_proj", "")
             key = (layer, {"q": "qkv", "k": "qkv", "v": "qkv", "gate": "gu", "up": "gu"}.get(kind, kind))
             if key == key_prev:
                 groups[-1].append(j)
             else:
                 groups.append([j])
             key_prev = key
-        return groups
+        return None if all(len(g) == 1 for g in groups) else groups
 
     def launch_step_grouped(self, k, stream):
         """One step with each group of independent linears in one grouped launch (no
@@ -653,8 +658,9 @@ def main(argv=None):
                    "ms_per_step": round(ms_grp / reps, 5),
                    "value": round(step_bytes[0] / (ms_grp / reps * 1e-3) / 1e9, 1),
                    "ungrouped_no_outputs_ms_per_step": round(ms_one / reps, 5),
-                   "how": "q/k/v and gate/up of each layer in one grinqh_decode_gemv_group launch; "
-                          "no optional outputs in either graph; pool entry 0"}
+                   "how": "the independent linears of a layer (q/k/v, gate/up) in one "
+                          "grinqh_decode_gemv_group launch; no optional outputs in either graph; "
+                          "pool entry 0"}
     two_kernel = {"ms_per_step": round(ms_two / reps, 5),
                   "value": round(step_bytes[0] / (ms_two / reps * 1e-3) / 1e9, 1),
                   "gemv_us_per_launch": round(gemv_launch_us, 3),
