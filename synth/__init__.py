@@ -202,13 +202,17 @@ def config1(bits=(2.0, 3.0, 4.0)):
 
 
 def config2():
-    """Uniform-width sweep on 4096 -> 14336 (Llama-3-8B up_proj shape)."""
+    """Uniform-width sweep on 4096 -> 14336 (Llama-3-8B up_proj shape): base widths 8,
+    4 (and a mix) and 6."""
     out = [Linear(f"up14336_u{b}", 4096, 14336, target_bits=None, uniform_b=b, config_id=2,
                   layer=0) for b in (2, 4, 6, 8)]
     out += [Linear(f"up14336_bmax4_u{b}", 4096, 14336, b_max=4, target_bits=None, uniform_b=b,
                    config_id=2, layer=1) for b in (2, 4)]
     out.append(Linear("up14336_bmax4_mix", 4096, 14336, b_max=4, target_bits=2.4, config_id=2,
                       layer=1))
+    # the 6-bit base width (GRINQH-6b) at uniform widths
+    out += [Linear(f"up14336_bmax6_u{b}", 4096, 14336, b_max=6, target_bits=None, uniform_b=b,
+                   config_id=2, layer=2) for b in (2, 4, 6)]
     return out
 
 

@@ -226,7 +226,7 @@ def test_qwen3_8b_projections(idx, path):
 
 
 @pytest.mark.slow
-@pytest.mark.parametrize("idx", range(7))
+@pytest.mark.parametrize("idx", range(len(synth.config2())))
 @pytest.mark.parametrize("path", PATHS)
 def test_uniform_sweep_llama_up_proj(idx, path):
     lin = synth.config2()[idx]
