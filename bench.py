@@ -484,13 +484,25 @@ def bits_fit(cases, specs):
 
 # ---- the oracle on the host cores (baseline only) --------------------------------
 
-def oracle_sample_run(spec, rank=0, seconds=10.0, outs_per_rep=None):
-    """Times the oracle's assign + lists + gemv on one linear of the workload.
-    Returns (GB/s-equivalent, threads, description)."""
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def oracle_sample_run(spec, rank=0, seconds=10.0, outs_per_rep=None, threads=None):
+    """Times the oracle's assign + lists + gemv on one linear of the workload, on
+    `threads` host threads (default: all).  Returns (GB/s-equivalent, threads,
+    description)."""
     import oracle
     case = synth.make_case(spec)
     planes = oracle.pack(case.q, spec.b_max)  # offline step, not timed
-    threads = oracle.max_threads()
+    threads = threads or oracle.max_threads()
     n_out = spec.d_out if outs_per_rep is None else outs_per_rep
     outs = None if outs_per_rep is None else np.arange(n_out, dtype=np.int32)
     t0 = time.perf_counter()
@@ -505,7 +517,8 @@ def oracle_sample_run(spec, rank=0, seconds=10.0, outs_per_rep=None):
             break
     dt = time.perf_counter() - t0
     desc = (f"oracle assign+lists+gemv on {spec.name} ({spec.d_in}->{spec.d_out}), "
-            f"{n_out} outputs per run, {reps} runs in {dt:.1f} s, OpenMP over outputs")
+            f"{n_out} outputs per run, {reps} runs in {dt:.1f} s, "
+            f"{'OpenMP over outputs' if threads > 1 else 'one thread'}")
     return moved / dt / 1e9, threads, desc
 
 
@@ -699,8 +712,10 @@ def main(argv=None):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         spec = next(s for s in specs if s.d_in * s.d_out == min(x.d_in * x.d_out for x in specs))
         v, threads, desc = oracle_sample_run(spec, seconds=10.0)
+        v1, _, desc1 = oracle_sample_run(spec, seconds=5.0, threads=1)
         cpu = {"value": round(v, 4), "unit": UNIT, "cores": threads, "kind": "oracle",
-               "sample": desc}
+               "sample": desc, "cpu_model": cpu_model(),
+               "single_thread": {"value": round(v1, 4), "sample": desc1}}
 
     if dist is not None:
         dist.barrier()
