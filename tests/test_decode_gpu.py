@@ -171,6 +171,7 @@ def test_split_k_wait_gives_up_and_reports_a_stale_arrival():
     [(1024, 4096, 8), (4096, 1024, 8)],                           # different d_in
     [(512, 1040, 6), (1024, 3072, 4), (256, 16, 2), (2048, 1024, 8)],  # mixed widths, a ragged unaligned layout
     [(1024, 2048, 8)],                                            # a group of one
+    [(256, 150 * 1024 + 16, 8), (512, 1024, 8)],                  # more tiles than CTAs; a one-CTA tile
 ])
 def test_grouped_launch_matches_the_oracle_per_linear(shapes):
     from input_adaptive_bit_b200 import (grinqh_check_device_error, grinqh_decode_gemv_group,
