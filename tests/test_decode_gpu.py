@@ -205,3 +205,24 @@ def test_decode_group_helper_of_the_layer_module():
     for (q, s, z, x, theta), y in zip(cases, ys):
         out = {"y": y.cpu().numpy().astype(np.float64)}
         check_y(out, oracle.pack(q, 8), s, z, x, oracle.assign(x, theta, 8), 8)
+
+
+
+def test_grouped_launch_with_an_explicit_phi_table():
+    from input_adaptive_bit_b200 import grinqh_decode_gemv_group, grinqh_group_workspace_bytes
+    q1, s1, z1, x1, th1 = cheap_case(40, 1024, 2048, 8)
+    q2, s2, z2, x2, th2 = cheap_case(41, 512, 1024, 6)
+    phi1 = np.array([0.0, 0.37, -1.25, 3.5, 0.0], np.float32)  # any table: levels 0..4
+    l1, l2 = GrinqhLinear(q1, s1, z1, 8), GrinqhLinear(q2, s2, z2, 6)
+    y1 = torch.empty(2048, dtype=torch.float32, device="cuda")
+    y2 = torch.empty(1024, dtype=torch.float32, device="cuda")
+    nbytes = grinqh_group_workspace_bytes()
+    ws = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
+    grinqh_decode_gemv_group([(l1.planes, l1.s, l1.z, to_dev(x1), to_dev(th1), to_dev(phi1), 1024, 2048, 8, y1),
+                              (l2.planes, l2.s, l2.z, to_dev(x2), to_dev(th2), None, 512, 1024, 6, y2)],
+                             ws, nbytes)
+    torch.cuda.synchronize()
+    check_y({"y": y1.cpu().numpy().astype(np.float64)}, oracle.pack(q1, 8), s1, z1, x1,
+            oracle.assign(x1, th1, 8), 8, phi=phi1)
+    check_y({"y": y2.cpu().numpy().astype(np.float64)}, oracle.pack(q2, 6), s2, z2, x2,
+            oracle.assign(x2, th2, 6), 6)

@@ -52,3 +52,27 @@ def test_matches_the_workspace_entry_points_on_two_calls_in_a_row():
         _, bound = oracle.gemv(planes_ref, s, z, x, b_host, 8, threads=oracle.max_threads())
         assert np.isfinite(a).all()
         assert (np.abs(a - b) <= REL * bound + ABS).all(), f"call {call} differs"
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("b_max", [4, 6])
+def test_smaller_base_widths(b_max):
+    assert torch.cuda.is_available()
+    g = np.random.default_rng(77 + b_max)
+    d_in, d_out = 1024, 2048
+    q = g.integers(0, 1 << b_max, size=(d_in, d_out), dtype=np.uint8)
+    s = (g.random((d_in // 128, d_out)) * 0.01 + 1e-4).astype(np.float16)
+    z = (-(g.random((d_in // 128, d_out)) * 0.5)).astype(np.float16)
+    lin = GrinqhLinear(q, s, z, b_max)
+    x = synth.activations(g, d_in)
+    fr = np.full(b_max // 2 + 1, 1.0 / (b_max // 2 + 1))
+    theta = synth.quantile_thresholds(np.abs(x.astype(np.float32)), fr)
+    y = torch.full((d_out,), float("nan"), dtype=torch.float32, device="cuda")
+    grinqh_decode_gemv_noalloc(lin.planes, lin.s, lin.z, torch.from_numpy(x).cuda(),
+                               torch.from_numpy(theta).cuda(), None, d_in, d_out, b_max, y)
+    torch.cuda.synchronize()
+    b_host = oracle.assign(x, theta, b_max)
+    y_ref, bound = oracle.gemv(oracle.pack(q, b_max), s, z, x, b_host, b_max,
+                               threads=oracle.max_threads())
+    a = y.cpu().numpy()
+    assert (np.abs(a - y_ref) <= REL * bound + ABS).all()
