@@ -183,6 +183,26 @@ size_t grinqh_group_workspace_bytes(void);
 int grinqh_decode_gemv_group(int n, const grinqh_linear *lins, void *ws, size_t ws_bytes,
                              void *stream);
 
+/* ---- Prefill GEMM (every row at the full width b_max) -------------------------
+ * The pages' other phase: for a block of T tokens every input channel runs at
+ * the base width, so all P planes are read and
+ *   Y[t][o] = sum_i X[t][i] * (s[g][o] * (q[i][o] + phi_P) + z[g][o]),  g = i/128,
+ * q the full b_max-bit code.  Each w_hat is rebuilt in fp32 and rounded once
+ * to fp16 (relative error <= 2^-11, inside the decode tolerance); the products
+ * run on the tensor cores with fp32 accumulation, and the d_in slices of the
+ * split-K grid are added into Y (so the last bits of Y depend on their order).
+ *   planes, s, z  the packed layer, as for grinqh_decode_gemv; d_out must be a
+ *                 multiple of 128 (GRINQH_ERR_UNSUPPORTED_SHAPE otherwise).
+ *   x             fp16 [T][d_in] (16-byte aligned), T in [1, 65536].
+ *   phi           fp32 [b_max/2 + 1] or NULL (phi_P = 0).
+ *   y             fp32 [T][d_out] out (cleared by the call, then accumulated).
+ *   ws            at least grinqh_prefill_workspace_bytes() bytes (its device
+ *                 error word; 4 if a wait on the tensor cores gave up). */
+size_t grinqh_prefill_workspace_bytes(void);
+int grinqh_prefill_gemm(const uint32_t *planes, const uint16_t *s, const uint16_t *z,
+                        const uint16_t *x, const float *phi, int T, int d_in, int d_out,
+                        int b_max, float *y, void *ws, size_t ws_bytes, void *stream);
+
 /* Reads and clears the device error word of `ws` (synchronises `stream`).
  * Returns GRINQH_OK, or GRINQH_ERR_DEVICE with the device code in
  * grinqh_last_error(). */

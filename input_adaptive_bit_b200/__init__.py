@@ -20,6 +20,7 @@ __all__ = [
     "grinqh_check_device_error", "grinqh_pack_dense4", "grinqh_dense4_workspace_bytes",
     "grinqh_gemv_dense4", "grinqh_decode_gemv", "grinqh_decode_gemv_noalloc",
     "grinqh_group_workspace_bytes", "grinqh_decode_gemv_group", "GrinqhLinearDesc", "MAX_GROUP",
+    "grinqh_prefill_workspace_bytes", "grinqh_prefill_gemm",
     "EXPORTS",
 ]
 
@@ -63,6 +64,8 @@ EXPORTS = {
     "grinqh_decode_gemv_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _P, _P]),
     "grinqh_group_workspace_bytes": (_Z, []),
     "grinqh_decode_gemv_group": (_I, [_I, _P, _P, _Z, _P]),
+    "grinqh_prefill_workspace_bytes": (_Z, []),
+    "grinqh_prefill_gemm": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _Z, _P]),
 }
 
 
@@ -193,3 +196,13 @@ def grinqh_decode_gemv_group(lins, ws, ws_bytes, stream=None):
                                   d_in, d_out, b_max, _ptr(y))
     _check(lib().grinqh_decode_gemv_group(len(lins), ctypes.cast(arr, ctypes.c_void_p), _ptr(ws),
                                           ws_bytes, _stream(stream)))
+
+
+def grinqh_prefill_workspace_bytes() -> int:
+    return lib().grinqh_prefill_workspace_bytes()
+
+
+def grinqh_prefill_gemm(planes, s, z, x, phi, T, d_in, d_out, b_max, y, ws, ws_bytes, stream=None):
+    """Y[T][d_out] = X[T][d_in] times the full-width w_hat (the prefill GEMM)."""
+    _check(lib().grinqh_prefill_gemm(_ptr(planes), _ptr(s), _ptr(z), _ptr(x), _ptr(phi), T, d_in,
+                                     d_out, b_max, _ptr(y), _ptr(ws), ws_bytes, _stream(stream)))

@@ -210,6 +210,35 @@ int grinqh_decode_gemv(const uint32_t *planes, const uint16_t *s, const uint16_t
                      "grinqh_decode_gemv launch");
 }
 
+size_t grinqh_prefill_workspace_bytes(void) { return grinqh::prefill_ws_bytes(); }
+
+int grinqh_prefill_gemm(const uint32_t *planes, const uint16_t *s, const uint16_t *z,
+                        const uint16_t *x, const float *phi, int T, int d_in, int d_out,
+                        int b_max, float *y, void *ws, size_t ws_bytes, void *stream) {
+  TRY(check_bmax(b_max));
+  TRY(check_din(d_in));
+  TRY(check_dout(d_out));
+  if (d_out % 128 != 0)
+    return fail(GRINQH_ERR_UNSUPPORTED_SHAPE,
+                "grinqh_prefill_gemm: d_out must be a multiple of 128 (got %d)", d_out);
+  if (T < 1 || T > 65536)
+    return fail(GRINQH_ERR_UNSUPPORTED_SHAPE, "grinqh_prefill_gemm: T must be in [1, 65536] (got %d)",
+                T);
+  TRY(check_ptr(planes, 16, "planes"));
+  TRY(check_ptr(s, 16, "s"));
+  TRY(check_ptr(z, 16, "z"));
+  TRY(check_ptr(x, 16, "x"));
+  if (phi) TRY(check_ptr(phi, 4, "phi"));
+  TRY(check_ptr(y, 4, "y"));
+  TRY(check_ptr(ws, 256, "ws"));
+  if (ws_bytes < grinqh::prefill_ws_bytes())
+    return fail(GRINQH_ERR_WORKSPACE_TOO_SMALL, "workspace of %zu bytes, prefill needs %zu",
+                ws_bytes, grinqh::prefill_ws_bytes());
+  return cuda_status(grinqh::launch_prefill(planes, s, z, x, phi, T, d_in, d_out, b_max, y, ws,
+                                            (cudaStream_t)stream),
+                     "grinqh_prefill_gemm launch");
+}
+
 size_t grinqh_group_workspace_bytes(void) { return grinqh::group_ws_bytes(); }
 
 int grinqh_decode_gemv_group(int n, const grinqh_linear *lins, void *ws, size_t ws_bytes,

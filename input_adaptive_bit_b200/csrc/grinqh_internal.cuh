@@ -25,6 +25,7 @@ constexpr int kDecodeMaxDin = 65536;            // largest d_in of the fused dec
 constexpr int kDevErrStreamMismatch = 1;  // gemv saw a unit stream of another d_in / b_max
 constexpr int kDevErrBadUnit = 2;         // a unit record outside [0, d_in) x [0, P) (skipped)
 constexpr int kDevErrSplitKTimeout = 3;   // decode: a split-K wait gave up (y of that tile is wrong)
+constexpr int kDevErrPrefillTimeout = 4;  // prefill: a wait on the tensor cores gave up
 
 // Workspace header (first 256 bytes of the workspace).
 struct WsHeader {
@@ -191,6 +192,10 @@ cudaError_t launch_decode(const uint32_t *planes, const uint16_t *s, const uint1
                           int32_t *counts, float *grp_sums, void *ws, cudaStream_t st);
 cudaError_t launch_decode_group(int n, const grinqh_linear *lins, void *ws, cudaStream_t st);
 size_t group_ws_bytes();
+cudaError_t launch_prefill(const uint32_t *planes, const uint16_t *s, const uint16_t *z,
+                           const uint16_t *x, const float *phi, int T, int d_in, int d_out,
+                           int b_max, float *y, void *ws, cudaStream_t st);
+size_t prefill_ws_bytes();
 cudaError_t launch_pack_dense4(const uint8_t *q4, int d_in, int d_out, uint32_t *w4,
                                cudaStream_t st);
 size_t dense4_ws_bytes(int d_in, int d_out);
