@@ -3,6 +3,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload qwen3-8b-proj|uniform-sweep|70b|llama3-8b-step|gate-3b]
+    python bench.py --workload prefill-qwen3-8b [--tokens T]
 
 A step is one pass of the whole decode path over one token's inputs for every
 linear of the workload: by default the fused grinqh_decode_gemv call per linear
@@ -22,6 +23,12 @@ step, divided by the device time of the step.  One JSON line is printed by
 rank 0.  With --gpus N > 1 (under torchrun) every rank runs its own replica of
 the workload (weak scaling, no collective on the data path); the step time is
 the max over ranks.
+
+--workload prefill-qwen3-8b times the other phase instead: a step is the
+prefill GEMM (grinqh_prefill_gemm, every row at the full width b_max = 8) of
+a block of T prompt tokens (default 128) through the same four Qwen3-8B
+projections; the value is TFLOP/s (2 T d_in d_out per linear) against the
+measured dense 16-bit tensor peak.
 """
 from __future__ import annotations
 
@@ -70,9 +77,11 @@ def parse_args(argv=None):
                     help="fused: grinqh_decode_gemv per linear; two: grinqh_assign + grinqh_gemv")
     ap.add_argument("--workload", default="qwen3-8b-proj",
                     choices=["qwen3-8b-proj", "uniform-sweep", "70b", "llama3-8b-step",
-                             "gate-3b"],
+                             "gate-3b", "prefill-qwen3-8b"],
                     help="gate-3b: the single gate_proj 4096->12288 GEMV at 3 bits of the "
                          "qwen3-8b-proj set (a small case for profiler captures)")
+    ap.add_argument("--tokens", type=int, default=128,
+                    help="prefill-qwen3-8b: prompt tokens per step (T)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-cases", action="store_true", help="skip the per-GEMV cold-L2 table")
     return ap.parse_args(argv)
@@ -522,6 +531,288 @@ def oracle_sample_run(spec, rank=0, seconds=10.0, outs_per_rep=None, threads=Non
     return moved / dt / 1e9, threads, desc
 
 
+# ---- prefill workload ------------------------------------------------------------------
+
+PREFILL_BMAX = 8
+PREFILL_SETS = 2  # distinct weight sets, alternated step by step
+PREFILL_SWEEP_T = (1, 16, 64, 128, 256, 512, 1024, 2048)
+
+
+def measured_tensor_peak(sustained: bool):
+    """Dense 16-bit tensor-core peak in TFLOP/s: the measured cuBLAS bf16 figure
+    (fp16 has the same nominal dense rate on B200, ratio 1)."""
+    key = "bf16_tflops_sustained" if sustained else "bf16_tflops"
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)[key]), "measured " + key
+    except Exception:
+        return (1400.0 if sustained else 1590.0), "fallback"
+
+
+def prefill_weights(g, d_in, d_out, b_max=PREFILL_BMAX):
+    """Random base codes and fp16 s, z for a prefill layer; the prefill GEMM does
+    the same work whatever the code values are."""
+    q = g.integers(0, 1 << b_max, size=(d_in, d_out), dtype=np.uint8)
+    s = (g.random((d_in // 128, d_out)) * 0.01 + 1e-4).astype(np.float16)
+    z = (-(g.random((d_in // 128, d_out)) * 0.5)).astype(np.float16)
+    return q, s, z
+
+
+class PrefillWorkload:
+    """PREFILL_SETS copies of the four Qwen3-8B projections (packed planes at
+    b_max 8), a token block X per input width, fp32 outputs and one step graph
+    per copy; plus fp16 dense weights of the same shapes for the cuBLAS
+    comparator."""
+
+    def __init__(self, T, device, rank):
+        import torch
+        from input_adaptive_bit_b200.layer import GrinqhLinear
+        self.torch, self.device, self.T = torch, device, T
+        self.shapes = list(synth.QWEN3_8B)
+        self.sets = []
+        for si in range(PREFILL_SETS):
+            layers = []
+            for li, (_, di, do) in enumerate(self.shapes):
+                q, s, z = prefill_weights(synth.rng(5, 100 * si + li, rank), di, do)
+                layers.append(GrinqhLinear(q, s, z, PREFILL_BMAX, device=device))
+                del q
+            self.sets.append(layers)
+        widths = sorted({di for _, di, _ in self.shapes})
+        g = synth.rng(5, 900, rank)
+        self.x_host = {d: torch.from_numpy(synth.prefill_tokens(g, T, d)).pin_memory()
+                       for d in widths}
+        self.x_dev = {d: h.to(device) for d, h in self.x_host.items()}
+        self.y_dev = [torch.zeros((T, do), dtype=torch.float32, device=device)
+                      for _, _, do in self.shapes]
+        self.y_host = [torch.zeros((T, do), dtype=torch.float32).pin_memory()
+                       for _, _, do in self.shapes]
+        self.stream = torch.cuda.Stream(device=device)
+        self.flops = sum(2 * T * di * do for _, di, do in self.shapes)
+        self.plane_bytes = sum(di * do * PREFILL_BMAX // 8 for _, di, do in self.shapes)
+        self.graphs = [self._capture(lambda k=k: self.body(k)) for k in range(PREFILL_SETS)]
+
+    def body(self, k):
+        for lin, (_, di, _), y in zip(self.sets[k], self.shapes, self.y_dev):
+            lin.prefill(self.x_dev[di], Y=y, stream=self.stream)
+
+    def _capture(self, fn):
+        torch, st = self.torch, self.stream
+        with torch.cuda.stream(st):
+            fn()  # first launches outside the capture (smem attributes)
+            st.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=st):
+                fn()
+        return g
+
+    def dense_graphs(self):
+        """cuBLAS fp16 X @ W on the same shapes (PREFILL_SETS weight copies)."""
+        torch = self.torch
+        ws = [[torch.randn((di, do), dtype=torch.float16, device=self.device) * 0.02
+               for _, di, do in self.shapes] for _ in range(PREFILL_SETS)]
+        outs = [torch.empty((self.T, do), dtype=torch.float16, device=self.device)
+                for _, _, do in self.shapes]
+
+        def body(k):
+            for w, (_, di, _), o in zip(ws[k], self.shapes, outs):
+                torch.mm(self.x_dev[di], w, out=o)
+
+        graphs = [self._capture(lambda k=k: body(k)) for k in range(PREFILL_SETS)]
+        return graphs, (ws, outs)
+
+
+def prefill_sweep(device, reps=10):
+    """The gate_proj shape (4096 -> 12288) at several token counts, cold L2: a
+    graph of reps x (256 MB read, call) minus a graph of reps x (256 MB read),
+    for grinqh_prefill_gemm and for cuBLAS fp16 on dense weights."""
+    import torch
+    from input_adaptive_bit_b200.layer import GrinqhLinear
+    di, do = 4096, 12288
+    q, s, z = prefill_weights(synth.rng(5, 950, 0), di, do)
+    lin = GrinqhLinear(q, s, z, PREFILL_BMAX, device=device)
+    del q
+    w16 = torch.randn((di, do), dtype=torch.float16, device=device) * 0.02
+    flush = L2Flush(torch, device)
+    st = torch.cuda.Stream(device=device)
+    t_flush = _graph_ms(torch, st, flush, reps) / reps
+    g = synth.rng(5, 951, 0)
+    rows = []
+    for T in PREFILL_SWEEP_T:
+        X = torch.from_numpy(synth.prefill_tokens(g, T, di)).to(device)
+        Y = torch.empty((T, do), dtype=torch.float32, device=device)
+        Yh = torch.empty((T, do), dtype=torch.float16, device=device)
+
+        def ours():
+            flush()
+            lin.prefill(X, Y=Y, stream=st)
+
+        def dense():
+            flush()
+            torch.mm(X, w16, out=Yh)
+
+        us = (_graph_ms(torch, st, ours, reps) / reps - t_flush) * 1e3
+        us_d = (_graph_ms(torch, st, dense, reps) / reps - t_flush) * 1e3
+        fl = 2.0 * T * di * do
+        rows.append({"T": T, "us": round(us, 2), "TFLOPs": round(fl / (us * 1e-6) / 1e12, 1),
+                     "plane_GBps": round(di * do / (us * 1e3), 1),
+                     "cublas_fp16_us": round(us_d, 2),
+                     "cublas_fp16_TFLOPs": round(fl / (us_d * 1e-6) / 1e12, 1),
+                     "time_vs_cublas": round(us / us_d, 3)})
+    return rows
+
+
+def oracle_prefill_sample(seconds=10.0, threads=None):
+    """The oracle's full-width GEMV of one token after another on q_proj
+    (4096 -> 4096).  Returns (TFLOP/s, threads, description)."""
+    import oracle
+    di, do = 4096, 4096
+    q, s, z = prefill_weights(synth.rng(5, 960, 0), di, do)
+    planes = oracle.pack(q, PREFILL_BMAX)  # offline step, not timed
+    X = synth.prefill_tokens(synth.rng(5, 961, 0), 64, di)
+    full = np.full(di, PREFILL_BMAX, np.uint8)
+    threads = threads or oracle.max_threads()
+    t0 = time.perf_counter()
+    n = 0
+    while True:
+        oracle.gemv(planes, s, z, X[n % len(X)], full, PREFILL_BMAX, threads=threads)
+        n += 1
+        if time.perf_counter() - t0 >= seconds:
+            break
+    dt = time.perf_counter() - t0
+    desc = (f"oracle full-width gemv of {n} tokens on q_proj (4096->4096) in {dt:.1f} s, "
+            f"{'OpenMP over outputs' if threads > 1 else 'one thread'}")
+    return 2.0 * di * do * n / dt / 1e12, threads, desc
+
+
+def run_prefill(args):
+    import torch
+    rank, world, dist = init_dist(torch)
+    device = torch.device("cuda", torch.cuda.current_device())
+    from input_adaptive_bit_b200 import lib
+    lib()  # fail loudly if the CUDA library is missing
+    T = args.tokens
+    wl = PrefillWorkload(T, device, rank)
+    props = torch.cuda.get_device_properties(device)
+    try:
+        gpu_id = "GPU-" + str(props.uuid)
+    except Exception:
+        gpu_id = None
+    sampler = ClockSampler(gpu_id)
+
+    def barrier():
+        torch.cuda.synchronize(device)
+        if dist is not None:
+            dist.barrier()
+
+    def run(graphs, i):
+        graphs[i % PREFILL_SETS].replay()
+
+    with torch.cuda.stream(wl.stream):
+        for i in range(args.warmup):
+            run(wl.graphs, i)
+    barrier()
+    sampler.start()
+    time.sleep(0.3)
+    barrier()
+    with torch.cuda.stream(wl.stream):
+        ms = device_time_ms(torch, wl.stream, lambda i: run(wl.graphs, i), args.steps)
+    barrier()
+    time.sleep(0.1)
+    clocks = ClockSampler.summarize(sampler.stop())
+    ms = max_over_ranks(dist, ms, device)
+    ms_step = ms / args.steps
+    value = world * wl.flops * args.steps / (ms * 1e-3) / 1e12
+
+    # cuBLAS fp16 on dense weights of the same shapes, same protocol
+    dgraphs, keep = wl.dense_graphs()
+    reps = max(20, min(1000, args.steps))
+    with torch.cuda.stream(wl.stream):
+        for i in range(3):
+            run(dgraphs, i)
+        ms_d = device_time_ms(torch, wl.stream, lambda i: run(dgraphs, i), reps)
+    ms_d = max_over_ranks(dist, ms_d, device) / reps
+    del dgraphs, keep
+
+    # end to end: pinned X H2D, the step, Y D2H, host sync, every step
+    k_e2e = max(10, min(args.steps, 200))
+    h2d = sum(h.numel() * 2 for h in wl.x_host.values())
+    d2h = sum(h.numel() * 4 for h in wl.y_host)
+
+    def e2e_step(i):
+        for d, h in wl.x_host.items():
+            wl.x_dev[d].copy_(h, non_blocking=True)
+        run(wl.graphs, i)
+        for yd, yh in zip(wl.y_dev, wl.y_host):
+            yh.copy_(yd, non_blocking=True)
+        wl.stream.synchronize()
+
+    barrier()
+    with torch.cuda.stream(wl.stream):
+        for i in range(3):
+            e2e_step(i)
+        t0 = time.perf_counter()
+        ms_e2e = device_time_ms(torch, wl.stream, e2e_step, k_e2e)
+        wall = (time.perf_counter() - t0) * 1e3
+    ms_e2e = max_over_ranks(dist, max(ms_e2e, wall), device)
+    e2e_value = world * wl.flops * k_e2e / (ms_e2e * 1e-3) / 1e12
+
+    sweep = None
+    if rank == 0 and not args.no_cases:
+        sweep = prefill_sweep(device)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, threads, desc = oracle_prefill_sample(10.0)
+        cpu = {"value": round(v, 6), "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+               "sample": desc, "cpu_model": cpu_model()}
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    peak, peak_kind = measured_tensor_peak(sustained=True)
+    burst, _ = measured_tensor_peak(sustained=False)
+    hbm, hbm_kind = measured_peaks()
+    achieved = wl.flops / (ms_step * 1e-3) / 1e12
+    line = {
+        "metric": "prefill GEMM TFLOP/s at full width b_max 8", "value": round(value, 1),
+        "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 5), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f16 x f16 -> f32", "data": "synthetic",
+        "config": {"workload": "prefill of a %d-token block through the qwen3-8b projections "
+                               "(q 4096x4096, gate/up 4096x12288, down 12288x4096), every row "
+                               "at b_max 8" % T,
+                   "tokens": T, "gemms_per_step": len(wl.shapes),
+                   "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2: steps alternate between %d copies of the "
+                         "weights, %d MB of planes in all; no flush" % (
+                             PREFILL_SETS, PREFILL_SETS * wl.plane_bytes // 2**20),
+                   "flops_per_step": wl.flops, "plane_bytes_per_step": wl.plane_bytes},
+        "roofline": {"bound": "tensor", "kernel": "prefill_kernel (grinqh_prefill_gemm)",
+                     "achieved": round(achieved, 1), "peak": peak, "peak_kind": peak_kind,
+                     "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                     "frac_of_burst": round(achieved / burst, 4), "traffic": None,
+                     "hbm_view": {"plane_GBps": round(wl.plane_bytes / (ms_step * 1e-3) / 1e9, 1),
+                                  "peak": hbm, "peak_kind": hbm_kind},
+                     "how": "2 T d_in d_out per linear over the step's device time; the "
+                            "step also holds each call's memset of Y"},
+        "cublas_fp16_dense": {"ms_per_step": round(ms_d, 5),
+                              "TFLOPs": round(wl.flops / (ms_d * 1e-3) / 1e12, 1),
+                              "time_ratio": round(ms_step / ms_d, 3),
+                              "how": "torch.mm on fp16 weights of the same shapes, "
+                                     "%d weight copies alternated" % PREFILL_SETS},
+        "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": int(h2d),
+                "d2h_bytes_per_step": int(d2h), "steps": k_e2e,
+                "how": "pinned X H2D + step graph + Y D2H + host sync, every step"},
+        "gpu_launches": len(wl.shapes) * args.steps,
+        "clocks": clocks,
+        "cpu_baseline": cpu,
+    }
+    if sweep is not None:
+        line["sweep_gate_4096x12288"] = sweep
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 # ---- main ------------------------------------------------------------------------------
 
 def max_over_ranks(dist, v: float, device) -> float:
@@ -546,32 +837,54 @@ def dist_env():
     return rank, world, local
 
 
+def init_dist(torch):
+    """(rank, world, torch.distributed or None); one process per GPU over NCCL."""
+    rank, world, local = dist_env()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+        return rank, world, dist
+    torch.cuda.set_device(0)
+    return rank, world, None
+
+
 def run_reference(args):
     rank, world, _ = dist_env()
     if rank != 0:
         return 0
-    specs = workload_specs(args.workload)
-    spec = min(specs, key=lambda s: s.d_in * s.d_out)
     # the whole run stays near two minutes whatever K and W are; every step does
     # at least one full sample
     budget = min(20.0, 120.0 / max(1, args.steps + args.warmup))
+    if args.workload == "prefill-qwen3-8b":
+        metric, unit, dtype = "prefill GEMM TFLOP/s at full width b_max 8", "TFLOP/s", "f64"
+        sample = lambda sec: oracle_prefill_sample(sec)  # noqa: E731
+        sampled = "q_proj 4096->4096"
+    else:
+        metric, unit, dtype = METRIC, UNIT, "f64"
+        spec = min(workload_specs(args.workload), key=lambda s: s.d_in * s.d_out)
+        sample = lambda sec: oracle_sample_run(spec, seconds=sec, outs_per_rep=512)  # noqa: E731
+        sampled = spec.name
     vals = []
     for _ in range(args.warmup):
-        oracle_sample_run(spec, seconds=budget / 4, outs_per_rep=512)
+        sample(budget / 4)
     t0 = time.perf_counter()
+    threads, desc = 0, ""
     for _ in range(args.steps):
-        v, threads, desc = oracle_sample_run(spec, seconds=budget, outs_per_rep=512)
+        v, threads, desc = sample(budget)
         vals.append(v)
     dt = time.perf_counter() - t0
     value = float(np.mean(vals)) if vals else 0.0
-    line = {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": UNIT,
+    line = {"impl": "reference", "metric": metric, "value": round(value, 6), "unit": unit,
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(1e3 * dt / max(1, args.steps), 1), "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": args.workload, "sampled_linear": spec.name},
-            "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": threads,
+            "scaling": "weak", "vs_baseline": None, "dtype": dtype, "data": "synthetic",
+            "config": {"workload": args.workload, "sampled_linear": sampled},
+            "cpu_baseline": {"value": round(value, 6), "unit": unit, "cores": threads,
                              "kind": "oracle", "sample": desc},
-            "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0,
+            "e2e": {"value": round(value, 6), "unit": unit, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -582,17 +895,10 @@ def main(argv=None):
     if args.impl == "reference":
         return run_reference(args)
 
+    if args.workload == "prefill-qwen3-8b":
+        return run_prefill(args)
     import torch
-    rank, world, local = dist_env()
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-    else:
-        dist = None
-        torch.cuda.set_device(0)
+    rank, world, dist = init_dist(torch)
     device = torch.device("cuda", torch.cuda.current_device())
 
     from input_adaptive_bit_b200 import lib

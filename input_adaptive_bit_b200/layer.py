@@ -11,7 +11,8 @@ import torch
 
 from . import (MAX_GROUP, grinqh_decode_gemv_group, grinqh_group_workspace_bytes,
                grinqh_assign, grinqh_decode_gemv, grinqh_gemv, grinqh_gemv_dense4, grinqh_pack,
-               grinqh_pack_dense4, grinqh_dense4_workspace_bytes, grinqh_workspace_bytes)
+               grinqh_pack_dense4, grinqh_dense4_workspace_bytes, grinqh_prefill_gemm,
+               grinqh_prefill_workspace_bytes, grinqh_workspace_bytes)
 
 GROUP = 128
 
@@ -50,6 +51,9 @@ class GrinqhLinear:
         self.ws_bytes = grinqh_workspace_bytes(self.d_in, self.d_out, self.b_max)
         self.ws = torch.zeros(self.ws_bytes, dtype=torch.uint8, device=self.device)
         self.y = torch.empty(self.d_out, dtype=torch.float32, device=self.device)
+        self.prefill_ws_bytes = grinqh_prefill_workspace_bytes()
+        self.prefill_ws = torch.zeros(max(self.prefill_ws_bytes, 256), dtype=torch.uint8,
+                                      device=self.device)
 
     def assign(self, x, theta, phi=None, stream=None):
         grinqh_assign(x, theta, self.d_in, self.b_max, phi, self.b, self.lists, self.counts,
@@ -71,6 +75,16 @@ class GrinqhLinear:
                            self.counts if o else None, self.grp_sums if o else None, self.ws,
                            self.ws_bytes, stream)
         return y
+
+    def prefill(self, X, phi=None, Y=None, stream=None):
+        """Y[T][d_out] (fp32) = X[T][d_in] (fp16) times W_hat at the full width b_max:
+        the prefill GEMM on the same packed planes."""
+        T = int(X.shape[0])
+        if Y is None:
+            Y = torch.empty((T, self.d_out), dtype=torch.float32, device=self.device)
+        grinqh_prefill_gemm(self.planes, self.s, self.z, X, phi, T, self.d_in, self.d_out,
+                            self.b_max, Y, self.prefill_ws, self.prefill_ws_bytes, stream)
+        return Y
 
     def __call__(self, x, theta, phi=None, y=None, stream=None):
         """x: fp16 [d_in] on the device; theta: fp32 [b_max/2] on the device."""

@@ -96,6 +96,13 @@ def activations(g: np.random.Generator, d_in: int, dist: str = "normal",
     return x.astype(np.float16)
 
 
+def prefill_tokens(g: np.random.Generator, T: int, d_in: int) -> np.ndarray:
+    """A block of T prompt tokens' inputs, fp16 [T][d_in]: each row drawn as
+    ``activations(g, d_in)``."""
+    return np.stack([activations(g, d_in) for _ in range(T)]) if T else \
+        np.zeros((0, d_in), np.float16)
+
+
 def quantile_thresholds(abs_pool: np.ndarray, fractions) -> np.ndarray:
     """Static Theta from |x| quantiles: theta_k = sorted(|x|)[floor(c_k * n)],
     c_k = fraction of channels below level k.  Returns fp32 [P]."""
