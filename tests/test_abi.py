@@ -170,3 +170,34 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(gq, "lib_path", str(tmp_path / "absent.so"))
     with pytest.raises(ImportError):
         gq.grinqh_version()
+
+
+def test_prefill_argument_checks():
+    # planes, s, z, x, phi, T, d_in, d_out, b_max, y, ws, ws_bytes, stream
+    ok = [FAKE, FAKE, FAKE, FAKE, None, 128, 4096, 4096, 8, FAKE, FAKE, 4096, None]
+    for k in (0, 1, 2, 3, 9, 10):  # every required pointer, null or misaligned
+        for bad_ptr in (None, FAKE + 2):
+            bad = list(ok)
+            bad[k] = bad_ptr
+            assert _status("grinqh_prefill_gemm", *bad) == gq.ERR_INVALID_ARG, (k, bad_ptr)
+    bad = list(ok)
+    bad[4] = FAKE + 2  # phi is fp32
+    assert _status("grinqh_prefill_gemm", *bad) == gq.ERR_INVALID_ARG
+    for T in (0, -1, 65537):
+        bad = list(ok)
+        bad[5] = T
+        assert _status("grinqh_prefill_gemm", *bad) == gq.ERR_UNSUPPORTED_SHAPE, T
+    bad = list(ok)
+    bad[7] = 4096 + 16  # a multiple of 16 but not of the 128-output tile
+    assert _status("grinqh_prefill_gemm", *bad) == gq.ERR_UNSUPPORTED_SHAPE
+    assert "128" in gq.lib().grinqh_last_error().decode()
+    bad = list(ok)
+    bad[6] = 4096 + 64  # d_in not a whole number of 128-row groups
+    assert _status("grinqh_prefill_gemm", *bad) == gq.ERR_UNSUPPORTED_SHAPE
+    bad = list(ok)
+    bad[8] = 5
+    assert _status("grinqh_prefill_gemm", *bad) == gq.ERR_INVALID_ARG
+    bad = list(ok)
+    bad[11] = gq.grinqh_prefill_workspace_bytes() - 1
+    assert _status("grinqh_prefill_gemm", *bad) == gq.ERR_WORKSPACE_TOO_SMALL
+    assert gq.grinqh_prefill_workspace_bytes() > 0
