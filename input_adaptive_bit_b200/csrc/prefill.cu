@@ -58,7 +58,8 @@ constexpr int kRowsPerBuilder = kPK * kPM / 16 / (32 * kBuildWarps);  // rows of
 static_assert(kRowsPerBuilder * 32 * kBuildWarps * 16 == kPK * kPM, "every (row, word) once");
 constexpr int kSP = 4;    // plane-word (and s, z) slots
 constexpr int kSX = 3;    // X slots
-constexpr int kPSpinLimit = 1 << 20;  // polls of one wait; after a timeout a thread stops waiting
+constexpr uint32_t kWaitHintNs = 1000000;  // suspend-time hint of one try_wait (1 ms)
+constexpr int kPSpinLimit = 1000;           // tries of one wait (~1 s); after a timeout a thread stops waiting
 
 // shared memory map (bytes)
 constexpr size_t kABuf = (size_t)kPM * kPK * 2;       // A tile, fp16, MN-major
@@ -92,15 +93,18 @@ __device__ __forceinline__ void cp_async16(void *dst, const void *src, int src_b
 __device__ __forceinline__ void mbar_init(uint64_t *bar, unsigned count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(smem_u32(bar)), "r"(count));
 }
+// Waits for the phase of the given parity.  Each try_wait may suspend the thread
+// for up to kWaitHintNs and returns as soon as the phase completes, so a waiting
+// warp does not take issue slots from the others; at most kPSpinLimit tries.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, unsigned parity) {
   const unsigned a = smem_u32(bar);
   for (int i = 0; i < kPSpinLimit; ++i) {
     unsigned done;
     asm volatile(
-        "{.reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+        "{.reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
         " selp.u32 %0, 1, 0, p;}\n"
         : "=r"(done)
-        : "r"(a), "r"(parity)
+        : "r"(a), "r"(parity), "r"(kWaitHintNs)
         : "memory");
     if (done) return true;
   }
