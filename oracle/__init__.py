@@ -172,6 +172,29 @@ def gemv(planes, s, z, x, b, b_max: int, phi=None, outs=None, threads: int = 1):
     return y, bound
 
 
+def union_widths(X, theta, b_max: int) -> np.ndarray:
+    """Small batch ("GRINQH: Graded Input-Based Quantization Hierarchy for
+    Efficient LLM Generation", Limitations and outlook: beyond batch 1 the
+    requests' active channels differ): every token t of X [B][d_in] gets its own
+    widths b^(t) = assign(x_t); a step that rebuilds each weight once for the
+    whole batch must read, for row i, the planes of u_i = max_t b_i^(t)."""
+    return np.max(np.stack([assign(x, theta, b_max) for x in np.atleast_2d(X)]), axis=0)
+
+
+def gemv_batch(planes, s, z, X, theta, b_max: int, phi=None, threads: int = 1):
+    """The small-batch decode step by its definition: y_t = W_hat(b^(t))^T x_t
+    for each token t, each with its own widths (same section as union_widths).
+    Returns (Y [B][d_out], bounds [B][d_out], widths [B][d_in])."""
+    X = np.atleast_2d(X)
+    bs = np.stack([assign(x, theta, b_max) for x in X])
+    ys, bounds = [], []
+    for x, b in zip(X, bs):
+        y, bound = gemv(planes, s, z, x, b, b_max, phi=phi, threads=threads)
+        ys.append(y)
+        bounds.append(bound)
+    return np.stack(ys), np.stack(bounds), bs
+
+
 def pack_dense4(q4) -> np.ndarray:
     q4 = np.ascontiguousarray(q4, np.uint8)
     d_in, d_out = q4.shape
