@@ -14,7 +14,10 @@ from input_adaptive_bit_b200.layer import GrinqhLinear
 pytestmark = pytest.mark.gpu
 
 
-def run_case(seed, T, d_in, d_out, b_max, phi=None):
+def run_case(seed, T, d_in, d_out, b_max, phi=None, tokens=None, outs=None):
+    """Runs the prefill GEMM on seeded inputs and compares the given tokens (default:
+    the first, the last and six random ones) on the given outputs (default: all)
+    with the oracle's full-width GEMV."""
     g = np.random.default_rng(seed)
     q = g.integers(0, 1 << b_max, size=(d_in, d_out), dtype=np.uint8)
     s = (g.random((d_in // 128, d_out)) * 0.01 + 1e-4).astype(np.float16)
@@ -29,15 +32,19 @@ def run_case(seed, T, d_in, d_out, b_max, phi=None):
     torch.cuda.synchronize()
     grinqh_check_device_error(ws)
     Yh = Y.cpu().numpy().astype(np.float64)
+    assert np.isfinite(Yh).all()
     planes = oracle.pack(q, b_max)
     full = np.full(d_in, b_max, np.uint8)
-    rows = sorted(set([0, T - 1] + list(g.integers(0, T, 6))))
-    for t in rows:
+    if tokens is None:
+        tokens = sorted(set([0, T - 1] + list(g.integers(0, T, 6))))
+    cols = np.arange(d_out) if outs is None else np.asarray(outs, np.int32)
+    for t in tokens:
         y_ref, bound = oracle.gemv(planes, s, z, X[t], full, b_max,
                                    phi=None if phi is None else np.asarray(phi, np.float64),
-                                   threads=oracle.max_threads())
-        ok = oracle.within_tolerance(Yh[t], y_ref, bound, REL, ABS)
-        assert ok.all(), (t, np.flatnonzero(~ok)[:5], Yh[t][~ok][:5], y_ref[~ok][:5])
+                                   outs=None if outs is None else cols, threads=oracle.max_threads())
+        got = Yh[t][cols]
+        ok = oracle.within_tolerance(got, y_ref, bound, REL, ABS)
+        assert ok.all(), (t, cols[~ok][:5], got[~ok][:5], y_ref[~ok][:5])
 
 
 @pytest.mark.parametrize("T,d_in,d_out,b_max", [
@@ -54,3 +61,24 @@ def test_prefill_matches_the_oracle_at_full_width(T, d_in, d_out, b_max):
 
 def test_prefill_with_an_explicit_phi_table():
     run_case(99, 20, 512, 256, 8, phi=[0.0, 0.1, -0.2, 0.3, 0.45])
+
+
+def test_prefill_with_many_chunks_per_cta():
+    # 16 tiles x 64 chunks = 1024 work units over the GPU's CTAs: every CTA runs
+    # pieces of several chunks (the accumulator carried across MMAs, the copy
+    # rings wrapping around) and ranges that cross from one tile into the next
+    run_case(5, 16, 8192, 2048, 8, tokens=[0, 7, 15])
+
+
+def test_prefill_with_many_chunks_per_cta_and_phi():
+    run_case(6, 24, 4096, 4096, 6, phi=[0.0, 0.2, -0.1, 0.3], tokens=[0, 11, 23])
+
+
+def test_prefill_at_the_benchmark_shape_on_sampled_outputs():
+    # the gate projection of the prefill benchmark (4096 -> 12288, a 128-token
+    # block, b_max 8), in the benchmark's launch configuration; 512 sampled
+    # outputs (the first and last tile included) of four tokens
+    g = np.random.default_rng(8)
+    outs = np.unique(np.concatenate([np.arange(128), np.arange(12288 - 128, 12288),
+                                     g.integers(0, 12288, 256)]))
+    run_case(7, 128, 4096, 12288, 8, tokens=[0, 1, 64, 127], outs=outs)
