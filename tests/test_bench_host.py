@@ -77,3 +77,41 @@ def test_reference_arm_only_rank0_prints(monkeypatch, capsys):
     for k in ("metric", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
               "scaling", "vs_baseline", "dtype", "data", "config"):
         assert k in line
+
+
+def test_prefill_reference_arm_reports_tflops(monkeypatch, capsys):
+    monkeypatch.setattr(bench, "oracle_prefill_sample",
+                        lambda seconds=10.0, threads=None: (0.0007, 8, "fake prefill sample"))
+    args = bench.parse_args(["--impl", "reference", "--workload", "prefill-qwen3-8b",
+                             "--steps", "2", "--warmup", "1"])
+    monkeypatch.setenv("RANK", "0")
+    monkeypatch.setenv("WORLD_SIZE", "1")
+    assert bench.run_reference(args) == 0
+    line = json.loads(capsys.readouterr().out.strip())
+    assert line["impl"] == "reference" and line["unit"] == "TFLOP/s"
+    assert line["metric"].startswith("prefill GEMM")
+    assert line["value"] == pytest.approx(0.0007)
+    assert line["e2e"]["unit"] == "TFLOP/s" and line["cpu_baseline"]["unit"] == "TFLOP/s"
+    assert line["config"]["workload"] == "prefill-qwen3-8b"
+
+
+def test_tensor_peak_reads_the_measured_file():
+    import json as _json
+    try:
+        with open(os.path.join(bench.ROOT, "MEASURED_PEAKS.json")) as f:
+            mp_ = _json.load(f)
+    except OSError:
+        mp_ = {}
+    for sustained, key, fallback in ((True, "bf16_tflops_sustained", 1400.0), (False, "bf16_tflops", 1590.0)):
+        if key in mp_:
+            assert bench.measured_tensor_peak(sustained) == (float(mp_[key]), "measured " + key)
+        else:
+            assert bench.measured_tensor_peak(sustained) == (fallback, "fallback")
+
+
+def test_prefill_weights_shapes_and_ranges():
+    import numpy as np
+    q, s, z = bench.prefill_weights(np.random.default_rng(0), 256, 128, 6)
+    assert q.shape == (256, 128) and q.dtype == np.uint8 and q.max() < 64
+    assert s.shape == z.shape == (2, 128) and s.dtype == z.dtype == np.float16
+    assert (s > 0).all() and (z <= 0).all()
