@@ -12,13 +12,16 @@
 //    a few tiles, and each (range, tile) piece adds its partial sums into Y,
 //    which the launcher clears first.
 //  * Warp roles, connected by full/empty mbarrier rings (no block-wide barrier
-//    inside the loop): warps 8-11 copy the plane words and s, z of a chunk
-//    into one of 4 slots with cp.async, warps 12-15 the X rows into one of 3
-//    slots, each arriving on the slot's "full" barrier when its copies land;
-//    warps 0-7 rebuild the chunk's A tile into one of 2 buffers and arrive on
-//    "A full"; warp 16 issues the MMAs and commits them to "A empty", "X slot
-//    empty" and, after the last chunk of a piece, "accumulator full", on which
-//    warps 0-7 run the piece's epilogue and then free the accumulator.
+//    inside the loop): warps 16-19 copy the plane words and s, z of a chunk
+//    into one of 4 slots with cp.async (lanes 2j and 2j+1 take the two halves
+//    of one 32-byte row segment, so every sector is one request), warps 20-23
+//    the X rows into one of 3 slots, each arriving on the slot's "full" barrier
+//    when its copies land; warps 0-15 rebuild the chunk's A tile into one of 2
+//    buffers and arrive on "A full"; warp 24 issues the MMAs and commits them
+//    to "A empty", "X slot empty" and, after the last chunk of a piece,
+//    "accumulator full", on which warps 0-15 run the piece's epilogue and then
+//    free the accumulator.  A waiting thread sleeps in mbarrier.try_wait until
+//    the phase completes.
 //  * Rebuild, about 2 logic ops and 1 fp16 op per weight: each thread takes 2
 //    rows of one 16-output plane word.  Per row it rotates plane p's word left
 //    by 2 (P-1-p), so that output j's digit of plane p sits at bit
