@@ -187,13 +187,12 @@ int grinqh_decode_gemv_group(int n, const grinqh_linear *lins, void *ws, size_t 
  * The pages' other phase: for a block of T tokens every input channel runs at
  * the base width, so all P planes are read and
  *   Y[t][o] = sum_i X[t][i] * (s[g][o] * (q[i][o] + phi_P) + z[g][o]),  g = i/128,
- * q the full b_max-bit code.  Each w_hat is the fp16 rounding of s q + c, one
- * fused fp16 multiply-add of the exact code, with c = z + s phi_P rounded to
- * fp16 (c = z when phi_P = 0, and then w_hat is the correctly rounded fp16 of
- * the exact value: relative error <= 2^-11, inside the decode tolerance); the
- * products run on the tensor cores with fp32 accumulation, and the partial sums
- * of the d_in ranges are added into Y (so the last bits of Y depend on their
- * order).
+ * q the full b_max-bit code.  Each w_hat is rounded once to fp16: one fused
+ * fp16 multiply-add s q + z of the exact code when phi_P = 0 (the correctly
+ * rounded value, relative error <= 2^-11, inside the decode tolerance), and
+ * fmaf(s, q + phi_P, z) in fp32 when an explicit phi_P != 0; the products run
+ * on the tensor cores with fp32 accumulation, and the partial sums of the d_in
+ * ranges are added into Y (so the last bits of Y depend on their order).
  *   planes, s, z  the packed layer, as for grinqh_decode_gemv; d_out must be a
  *                 multiple of 128 (GRINQH_ERR_UNSUPPORTED_SHAPE otherwise).
  *   x             fp16 [T][d_in] (16-byte aligned), T in [1, 65536].

@@ -30,8 +30,9 @@
 //    r+8, r+12 as the four bytes of one register.  Byte permutes pair the
 //    codes of outputs (2c, 2c+1) under the fp16 exponent of 1024, so each half
 //    is exactly 1024 + q; one fp16 subtract (exact) and one fp16 FMA give
-//    w_hat = RN16(s q + c) with c = z + s phi_P (c = z when phi_P = 0, and then
-//    w_hat is the correctly rounded fp16 of the exact value).
+//    w_hat = RN16(s q + z), the correctly rounded fp16 of the exact value
+//    (phi_P = 0, the default).  With an explicit phi_P != 0 the FMA runs in
+//    fp32, fmaf(s, q + phi_P, z), rounded once to fp16.
 //  * The A tile is stored MN-major (8 consecutive outputs per 16-byte row of a
 //    core matrix), so a thread writes whole 16-byte rows; a warp's lanes cover
 //    the 8 rows of a core matrix and the stores are free of bank conflicts.  The
@@ -158,6 +159,19 @@ __device__ __forceinline__ uint32_t h2_sub_fma(uint32_t h, uint32_t s2, uint32_t
   return *reinterpret_cast<const uint32_t *>(&w);
 }
 
+// The same with an explicit phi_P != 0: fmaf(s, q + phi_P, z) in fp32, rounded
+// once to fp16.  (Folding phi_P into an fp16 offset z + s phi_P would round it,
+// and that one error would land on every weight of the group: where s q + z
+// nearly cancels it exceeds the per-weight 2^-11.)
+__device__ __forceinline__ uint32_t h2_sub_fma_phi(uint32_t h, uint32_t s2, uint32_t z2, float phi) {
+  const __half2 q = __hsub2(*reinterpret_cast<const __half2 *>(&h), __half2half2(__ushort_as_half(0x6400)));
+  const float2 qf = __half22float2(q);
+  const float2 sf = __half22float2(*reinterpret_cast<const __half2 *>(&s2));
+  const float2 zf = __half22float2(*reinterpret_cast<const __half2 *>(&z2));
+  const __half2 w = __floats2half2_rn(fmaf(sf.x, qf.x + phi, zf.x), fmaf(sf.y, qf.y + phi, zf.y));
+  return *reinterpret_cast<const uint32_t *>(&w);
+}
+
 // Codes (2P bits) of outputs r, r + 4, r + 8, r + 12 of a 16-output plane word
 // group, one per byte, from the P words rotated as described above.
 template <int P>
@@ -244,7 +258,7 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_kernel(const __grid_cons
         const unsigned char *slot = smem + kOffPlanes + (size_t)sp * kPlaneSlot;
         const uint16_t *sz = reinterpret_cast<const uint16_t *>(smem + kOffSz + (size_t)sp * kSzSlot);
         unsigned char *abuf = smem + kOffA + (size_t)(ci & 1) * kABuf;
-        uint32_t s2[8], c2[8];
+        uint32_t s2[8], z2[8];  // half2 s and z of outputs (2e, 2e + 1)
         {
           const uint4 sa = *reinterpret_cast<const uint4 *>(sz + 16 * wc);
           const uint4 sb = *reinterpret_cast<const uint4 *>(sz + 16 * wc + 8);
@@ -255,13 +269,7 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_kernel(const __grid_cons
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
             s2[e] = sv[e];
-            c2[e] = zv[e];
-            if (phiP != 0.0f) {
-              const float2 fs = __half22float2(*reinterpret_cast<const __half2 *>(&sv[e]));
-              const float2 fz = __half22float2(*reinterpret_cast<const __half2 *>(&zv[e]));
-              const __half2 c = __floats2half2_rn(fmaf(fs.x, phiP, fz.x), fmaf(fs.y, phiP, fz.y));
-              c2[e] = *reinterpret_cast<const uint32_t *>(&c);
-            }
+            z2[e] = zv[e];
           }
         }
 #pragma unroll
@@ -288,8 +296,13 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_kernel(const __grid_cons
           h[3] = prmt(u23a, K64, 0x4342u);
           h[5] = prmt(u23b, K64, 0x4140u);
           h[7] = prmt(u23b, K64, 0x4342u);
+          if (phiP == 0.0f) {
 #pragma unroll
-          for (int e = 0; e < 8; ++e) h[e] = h2_sub_fma(h[e], s2[e], c2[e]);
+            for (int e = 0; e < 8; ++e) h[e] = h2_sub_fma(h[e], s2[e], z2[e]);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) h[e] = h2_sub_fma_phi(h[e], s2[e], z2[e], phiP);
+          }
           unsigned char *dst = abuf + (k & 7) * 16 + (k >> 3) * 2048 + (2 * wc) * 128;
           *reinterpret_cast<uint4 *>(dst) = make_uint4(h[0], h[1], h[2], h[3]);
           *reinterpret_cast<uint4 *>(dst + 128) = make_uint4(h[4], h[5], h[6], h[7]);

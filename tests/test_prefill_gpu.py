@@ -82,3 +82,30 @@ def test_prefill_at_the_benchmark_shape_on_sampled_outputs():
     outs = np.unique(np.concatenate([np.arange(128), np.arange(12288 - 128, 12288),
                                      g.integers(0, 12288, 256)]))
     run_case(7, 128, 4096, 12288, 8, tokens=[0, 1, 64, 127], outs=outs)
+
+
+def test_prefill_explicit_phi_where_the_offset_cancels_the_codes():
+    # codes clustered at 128 with z = -128 s, so s q + z nearly cancels, and an
+    # explicit phi_P = 0.45: the rebuild must not round z + s phi_P to fp16 (that
+    # one error, shared by a group's weights, measures 1.4x the tolerance here)
+    g = np.random.default_rng(11)
+    T, d_in, d_out = 8, 2048, 256
+    q = np.clip(np.round(g.normal(128, 2, size=(d_in, d_out))), 0, 255).astype(np.uint8)
+    s = np.full((d_in // 128, d_out), 0.01, np.float16)
+    z = (-(s.astype(np.float64) * 128)).astype(np.float16)
+    X = g.standard_normal((T, d_in)).astype(np.float16)
+    phi = np.array([0.0, 0.1, -0.2, 0.3, 0.45])
+    lin = GrinqhLinear(q, s, z, 8)
+    Y = torch.full((T, d_out), float("nan"), dtype=torch.float32, device="cuda")
+    ws = torch.zeros(max(grinqh_prefill_workspace_bytes(), 256), dtype=torch.uint8, device="cuda")
+    grinqh_prefill_gemm(lin.planes, lin.s, lin.z, to_dev(X), to_dev(phi.astype(np.float32)), T, d_in, d_out,
+                        8, Y, ws, ws.numel())
+    torch.cuda.synchronize()
+    grinqh_check_device_error(ws)
+    Yh = Y.cpu().numpy().astype(np.float64)
+    planes = oracle.pack(q, 8)
+    full = np.full(d_in, 8, np.uint8)
+    for t in range(T):
+        y_ref, bound = oracle.gemv(planes, s, z, X[t], full, 8, phi=phi, threads=oracle.max_threads())
+        ok = oracle.within_tolerance(Yh[t], y_ref, bound, REL, ABS)
+        assert ok.all(), (t, np.flatnonzero(~ok)[:5])
