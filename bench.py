@@ -55,14 +55,12 @@ N_POOL = 8
 FALLBACK_HBM_GBS = 6650.0
 
 # DRAM bytes (read + write) per launch of the dominant kernel on the
-# qwen3-8b-proj step, from one ncu capture (profiles/), keyed by the SHA-256 of
-# the kernel source it was taken on: after any change to the kernel the figure
-# no longer applies and the bench reports null.
+# qwen3-8b-proj step, from one ncu launch-list capture of this workload, keyed by
+# the SHA-256 of the kernel source it was taken on: after any change to the
+# kernel the figure no longer applies and the bench reports null.
 NCU_TRAFFIC = {
-    # gemv.cu, grinqh_gemv (profiles/grinqh_gemv_qwen3-8b-proj_launches.md)
+    # gemv.cu, grinqh_gemv
     "84585736bc0dc9cf2ac9f0a4738586346a63ac0a4e44acbdc753bb3917df6db4": 17150844,
-    # decode.cu, grinqh_decode_gemv (profiles/decode_kernel_qwen3-8b-proj_launches.md)
-    "3b99529ba0960d7a26a4dd1bbdabdf74e36c38bd2fd67450277be62133263a3e": 17112247,
 }
 KERNEL_SOURCE = {"fused": "decode.cu", "two": "gemv.cu"}
 
@@ -489,6 +487,175 @@ def bits_fit(cases, specs):
     r2 = 1.0 - float(np.sum((t - (a + c * b)) ** 2)) / float(np.sum((t - t.mean()) ** 2))
     return {"us_per_bit": round(float(c), 3), "us_at_0_bits": round(float(a), 3),
             "r2": round(r2, 4), "points": [[int(x), round(float(y), 2)] for x, y in pts]}
+
+
+def uniform_sweep_fit(device, reps=20):
+    """Latency of the fused decode GEMV on the Llama-3-8B up_proj shape (4096 ->
+    14336, b_max 8) with every row at the same width b in {2, 4, 6, 8}, cold L2,
+    its least-squares fit against b, and the in-library dense 4-bit GEMV of the
+    same shape (the same bytes as b = 4)."""
+    import torch
+    from input_adaptive_bit_b200.layer import Dense4Linear, GrinqhLinear
+    spec = next(s for s in synth.config2() if s.b_max == 8)
+    W = synth.gaussian_weights(synth.rng(spec.config_id, spec.layer, 0), spec.d_in, spec.d_out)
+    q, s, z = synth.rtn_quantize(W, 8)
+    lin = GrinqhLinear(q, s, z, 8, device=device)
+    q4, s4, z4 = synth.rtn_quantize(W, 4)
+    d4 = Dense4Linear(q4, s4, z4, device=device)
+    del W, q, q4
+    x = torch.from_numpy(synth.make_x(spec, 0)).to(device)
+    y = torch.empty(spec.d_out, dtype=torch.float32, device=device)
+    flush = L2Flush(torch, device)
+    st = torch.cuda.Stream(device=device)
+    t_flush = _graph_ms(torch, st, flush, reps) / reps
+    pts = []
+    for b in (2, 4, 6, 8):
+        th = torch.from_numpy(synth.uniform_thresholds(b, 8)).to(device)
+
+        def call(th=th):
+            flush()
+            lin.decode(x, th, y=y, outputs=False, stream=st)
+
+        us = (_graph_ms(torch, st, call, reps) / reps - t_flush) * 1e3
+        nbytes = min_bytes(np.full(spec.d_in, b, np.uint8), spec.d_out)
+        pts.append((b, us, nbytes))
+
+    def dense():
+        flush()
+        d4(x, y=y, stream=st)
+
+    us_d4 = (_graph_ms(torch, st, dense, reps) / reps - t_flush) * 1e3
+    bits = np.array([p[0] for p in pts], np.float64)
+    t = np.array([p[1] for p in pts], np.float64)
+    c, a = np.polyfit(bits, t, 1)
+    r2 = 1.0 - float(np.sum((t - (a + c * bits)) ** 2)) / float(np.sum((t - t.mean()) ** 2))
+    d4_bytes = spec.d_in * spec.d_out // 2 + 4 * spec.d_out * (spec.d_in // 128) + 2 * spec.d_in \
+        + 4 * spec.d_out
+    return {"shape": "4096x14336 (b_max 8, every row at width b, cold L2)",
+            "us_per_bit": round(float(c), 3), "us_at_0_bits": round(float(a), 3),
+            "r2": round(r2, 4),
+            "points": [{"bits": b, "us": round(u, 2), "GBps": round(n / (u * 1e3), 1)}
+                       for b, u, n in pts],
+            "dense4_us": round(us_d4, 2), "dense4_GBps": round(d4_bytes / (us_d4 * 1e3), 1),
+            "time_4bit_vs_dense4": round(pts[1][1] / us_d4, 3)}
+
+
+def seventy_b_pair(device, peak, n_pool=64, reps=4):
+    """The 70B-class pair at 3 effective bits (8192 -> 28672 and 28672 -> 8192,
+    Student-t x, Theta from 128 pooled calibration draws): fused decode GEMVs
+    alternating between the two layers, a fresh x from a pool of n_pool per call
+    (so the active rows change every call); 470 MB of planes, no flush."""
+    import torch
+    from input_adaptive_bit_b200.layer import GrinqhLinear
+    specs = [s for s in synth.config3() if s.target_bits == 3.0]
+    layers, thetas, pools = [], [], []
+    for spec in specs:
+        W = synth.gaussian_weights(synth.rng(spec.config_id, spec.layer, 0), spec.d_in, spec.d_out)
+        q, s, z = synth.rtn_quantize(W, 8)
+        del W
+        layers.append(GrinqhLinear(q, s, z, 8, device=device))
+        del q
+        x0 = synth.activations(synth.rng(spec.config_id, spec.layer, 0), spec.d_in, spec.dist)
+        thetas.append(torch.from_numpy(synth.make_theta(spec, x0)).to(device))
+        pools.append(torch.from_numpy(np.stack([synth.make_x(spec, k) for k in range(n_pool)]))
+                     .to(device))
+    ys = [torch.empty(spec.d_out, dtype=torch.float32, device=device) for spec in specs]
+    st = torch.cuda.Stream(device=device)
+    # algorithmic bytes of every (layer, pool entry): widths from the kernel's own b output
+    nbytes = [[0] * n_pool for _ in specs]
+    eff = [[0.0] * n_pool for _ in specs]
+    with torch.cuda.stream(st):
+        for j, (lin, spec) in enumerate(zip(layers, specs)):
+            for k in range(n_pool):
+                lin.decode(pools[j][k], thetas[j], y=ys[j], stream=st)
+                st.synchronize()
+                b = lin.b.cpu().numpy()
+                nbytes[j][k] = min_bytes(b, spec.d_out)
+                eff[j][k] = float(b.mean())
+
+    def body():
+        for k in range(n_pool):
+            for j, lin in enumerate(layers):
+                lin.decode(pools[j][k], thetas[j], y=ys[j], outputs=False, stream=st)
+
+    ms = _graph_ms(torch, st, body, 1)  # one replay = 2 n_pool GEMVs
+    for _ in range(reps - 1):
+        ms = min(ms, _graph_ms(torch, st, body, 1))
+    total = sum(sum(v) for v in nbytes)
+    us = ms * 1e3 / (2 * n_pool)
+    gbps = total / (ms * 1e-3) / 1e9
+    out = {"shapes": "8192x28672 and 28672x8192 alternating, 3 effective bits (target), "
+                     "Student-t x, a fresh x per call from a pool of %d" % n_pool,
+           "us_per_gemv": round(us, 2), "GBps": round(gbps, 1),
+           "frac_of_hbm": round(gbps / peak, 4),
+           "eff_bits": {spec.name: round(float(np.mean(e)), 3) for spec, e in zip(specs, eff)},
+           "eff_bits_range": [round(min(min(e) for e in eff), 3), round(max(max(e) for e in eff), 3)]}
+    del layers, pools
+    torch.cuda.empty_cache()
+    return out
+
+
+def small_batch_sweep(device, reps=20, batches=(2, 4, 8)):
+    """The small-batch decode step (grinqh_decode_gemv_batch) on the gate_proj shape
+    (4096 -> 12288, b_max 8, Theta for 3 effective bits): B tokens, each its own
+    seeded x, cold L2.  Bytes are the union's: planes of u_i = max_t b_t(i), s/z of
+    groups with an active row, B inputs and B outputs."""
+    import torch
+    from input_adaptive_bit_b200 import grinqh_batch_workspace_bytes, grinqh_decode_gemv_batch
+    from input_adaptive_bit_b200.layer import GrinqhLinear
+    spec = next(s for s in synth.config1() if s.name == "gate_proj@3b")
+    W = synth.gaussian_weights(synth.rng(spec.config_id, spec.layer, 0), spec.d_in, spec.d_out)
+    q, s, z = synth.rtn_quantize(W, 8)
+    del W
+    lin = GrinqhLinear(q, s, z, 8, device=device)
+    del q
+    calib = synth.Linear(spec.name, spec.d_in, spec.d_out, 8, spec.target_bits, None, spec.dist,
+                         spec.config_id, spec.layer, calib_draws=128)
+    x0 = synth.activations(synth.rng(spec.config_id, spec.layer, 0), spec.d_in)
+    theta = torch.from_numpy(synth.make_theta(calib, x0)).to(device)
+    nws = grinqh_batch_workspace_bytes()
+    ws = torch.zeros(nws, dtype=torch.uint8, device=device)
+    flush = L2Flush(torch, device)
+    st = torch.cuda.Stream(device=device)
+    t_flush = _graph_ms(torch, st, flush, reps) / reps
+    rows = []
+    x1 = torch.from_numpy(synth.make_x(spec, 0)).to(device)
+    y1 = torch.empty(spec.d_out, dtype=torch.float32, device=device)
+
+    def one():
+        flush()
+        lin.decode(x1, theta, y=y1, outputs=False, stream=st)
+
+    us1 = (_graph_ms(torch, st, one, reps) / reps - t_flush) * 1e3
+    lin.decode(x1, theta, y=y1, stream=st)
+    st.synchronize()
+    b1 = lin.b.cpu().numpy()
+    rows.append({"B": 1, "us": round(us1, 2), "union_eff_bits": round(float(b1.mean()), 3),
+                 "GBps": round(min_bytes(b1, spec.d_out) / (us1 * 1e3), 1),
+                 "kernel": "grinqh_decode_gemv"})
+    for B in batches:
+        X = torch.from_numpy(np.stack([synth.make_x(spec, k) for k in range(B)])).to(device)
+        Y = torch.empty((B, spec.d_out), dtype=torch.float32, device=device)
+        u = torch.empty(spec.d_in, dtype=torch.uint8, device=device)
+        with torch.cuda.stream(st):
+            grinqh_decode_gemv_batch(lin.planes, lin.s, lin.z, X, theta, None, B, spec.d_in,
+                                     spec.d_out, 8, Y, u, ws, nws, stream=st)
+        st.synchronize()
+        un = u.cpu().numpy()
+
+        def call(X=X, Y=Y, B=B):
+            flush()
+            grinqh_decode_gemv_batch(lin.planes, lin.s, lin.z, X, theta, None, B, spec.d_in,
+                                     spec.d_out, 8, Y, None, ws, nws, stream=st)
+
+        us = (_graph_ms(torch, st, call, reps) / reps - t_flush) * 1e3
+        nbytes = min_bytes(un, spec.d_out) + (B - 1) * (2 * spec.d_in + 4 * spec.d_out)
+        rows.append({"B": B, "us": round(us, 2), "union_eff_bits": round(float(un.mean()), 3),
+                     "GBps": round(nbytes / (us * 1e3), 1),
+                     "tokens_per_s": round(B / (us * 1e-6), 1),
+                     "kernel": "grinqh_decode_gemv_batch"})
+    return {"shape": "gate_proj 4096x12288 at 3 effective bits per token (b_max 8), cold L2",
+            "points": rows}
 
 
 # ---- the oracle on the host cores (baseline only) --------------------------------
@@ -1008,11 +1175,20 @@ def main(argv=None):
     e2e_bytes = sum(step_bytes[i % N_POOL] for i in range(k_e2e))
     e2e_value = whole_job_gbps(world, e2e_bytes, ms_e2e)
 
+    planes_mb = sum(lin.planes.numel() * 4 for lin in wl.layers) // 2**20
     cases = None
     dense4 = None
+    sweep_fit = seventy = small_batch = None
     if not args.no_cases and rank == 0:
         cases = cold_case_times(wl)
         dense4 = dense4_times(wl)
+        if args.workload == "qwen3-8b-proj":
+            peak_hbm, _ = measured_peaks()
+            del wl
+            torch.cuda.empty_cache()
+            sweep_fit = uniform_sweep_fit(device)
+            seventy = seventy_b_pair(device, peak_hbm)
+            small_batch = small_batch_sweep(device)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -1040,7 +1216,7 @@ def main(argv=None):
                    "l2": "inputs larger than L2: each step reads ~%d MB of planes from %d MB of "
                          "distinct packed weights; no flush" % (
                              gemv_bytes[0] // 2**20,
-                             sum(l.planes.numel() * 4 for l in wl.layers) // 2**20),
+                             planes_mb),
                    "eff_bits": [round(e, 3) for e in eff_bits],
                    "us_per_gemv": round(ms * 1e3 / (args.steps * n_gemv), 3),
                    "bytes_per_step": int(np.mean(step_bytes))},
@@ -1067,6 +1243,12 @@ def main(argv=None):
         fit = bits_fit(cases, specs)
         if fit is not None:
             line["latency_vs_bits"] = fit
+    if sweep_fit is not None:
+        line["latency_vs_bits"] = sweep_fit
+    if seventy is not None:
+        line["seventy_b_class"] = seventy
+    if small_batch is not None:
+        line["small_batch"] = small_batch
     print(json.dumps(line), flush=True)
     return 0
 

@@ -142,9 +142,16 @@ int grinqh_gemv(const uint32_t *planes, const uint16_t *s, const uint16_t *z,
  * phi before waiting for that kernel; x, planes, s and z are read only after
  * the wait, and every output is written after it.  So theta and phi must not
  * be written by the kernel launched immediately before this call on the same
- * stream (a copy, an event or any other kernel in between lifts this).  The
- * split-K arrival wait does not give up on a correct launch; if it does (after
- * 2^20 polls, a fraction of a second) it sets the device error word to 3. */
+ * stream (a copy, an event or any other kernel in between lifts this).
+ * Device errors (grinqh_check_device_error): 3 if a split-K share was about to
+ * be summed with a partial sum missing, which happens only when the
+ * workspace's arrival words were not left zeroed (where a share has at most 32
+ * partial sums the call sees who is missing, waits for them, writes the right
+ * y and leaves the word zeroed); 5 if a wait inside the
+ * kernel's copy/MMA pipeline gave up (about a second; never on a correct
+ * launch), in which case y is not valid.  No CTA waits for another CTA outside
+ * its thread-block cluster, so the result does not depend on how many of the
+ * launch's CTAs the GPU runs at the same time. */
 int grinqh_decode_gemv(const uint32_t *planes, const uint16_t *s, const uint16_t *z,
                        const uint16_t *x, const float *theta, const float *phi, int d_in,
                        int d_out, int b_max, float *y, uint8_t *b, int32_t *lists,
@@ -182,6 +189,35 @@ typedef struct grinqh_linear {
 size_t grinqh_group_workspace_bytes(void);
 int grinqh_decode_gemv_group(int n, const grinqh_linear *lins, void *ws, size_t ws_bytes,
                              void *stream);
+
+/* ---- Small-batch decode (B <= 8 tokens sharing one read of the planes) --------
+ * GRINQH notes, "Limitations and outlook": beyond batch 1 the requests' active
+ * channels differ.  Every token t of the batch gets its own widths
+ * b_t(i) = 2 #{k : theta_k <= |x_t(i)|} and its own
+ *   y[t][o] = sum over i with b_t(i) > 0 of x[t][i] * w_hat_t(i, o),
+ *   w_hat_t(i, o) = s[g][o] * (Q_t(i, o) + phi_{b_t(i)/2}) + z[g][o],
+ * exactly what grinqh_decode_gemv computes for that token alone (within the
+ * rounding of a different summation order).  Row i's planes are read once, for
+ * the largest width any token gives it, and each field is decoded once.
+ *   planes, s, z  the packed layer, as for grinqh_decode_gemv.
+ *   x             fp16 [B][d_in], row t the input of token t (16-byte aligned).
+ *   theta, phi    as for grinqh_assign (one threshold set for the batch).
+ *   B             1 .. GRINQH_MAX_BATCH tokens.
+ *   y             fp32 [B][d_out] out; every element is written.
+ *   u             uint8 [d_in] out, or NULL: the union widths u_i = max_t b_t(i)
+ *                 (the planes read for row i), bit-exact.
+ *   ws            at least grinqh_batch_workspace_bytes() bytes, zero-filled once
+ *                 after allocation and left zeroed by every call; not shared
+ *                 with a concurrent call.
+ * Limits: d_in <= 65536.  Deterministic.  Launch overlap and device errors as
+ * for grinqh_decode_gemv (theta and phi are read before the wait on the kernel
+ * launched just before). */
+#define GRINQH_MAX_BATCH 8
+size_t grinqh_batch_workspace_bytes(void);
+int grinqh_decode_gemv_batch(const uint32_t *planes, const uint16_t *s, const uint16_t *z,
+                             const uint16_t *x, const float *theta, const float *phi, int B,
+                             int d_in, int d_out, int b_max, float *y, uint8_t *u, void *ws,
+                             size_t ws_bytes, void *stream);
 
 /* ---- Prefill GEMM (every row at the full width b_max) -------------------------
  * The pages' other phase: for a block of T tokens every input channel runs at
@@ -229,23 +265,38 @@ int grinqh_gemv_dense4(const uint32_t *w4, const uint16_t *s, const uint16_t *z,
  * every byte of device memory and only hands its plug-ins streams and tensors,
  * or a latency-critical path that must never enter the allocator.  It runs
  * the fused decode kernel (grinqh_decode_gemv without its optional outputs),
- * keeping its split-K scratch in a fixed array (about 2.2 MB) that the library
- * reserves on every GPU that loads it and holds until exit; it calls no
+ * keeping its split-K state (partial sums and arrival words) and its device
+ * error word in a fixed array of about 1.2 MB that the library reserves
+ * on every GPU that loads it and holds until exit; it calls no
  * cudaMalloc/cudaFree.
  *   planes, s, z  the packed layer (as for grinqh_gemv); x, theta, phi as for
  *                 grinqh_assign; y fp32 [d_out] out.
- *   Limits: d_in <= 32768 and d_out <= 32768, on top of the usual shape rules;
- *   larger shapes return GRINQH_ERR_UNSUPPORTED_SHAPE with a message.
+ *   Limits: those of grinqh_decode_gemv (d_in <= 65536); larger shapes return
+ *   GRINQH_ERR_UNSUPPORTED_SHAPE with a message, and nothing is queued on any
+ *   failed call.  The array holds the split-K state of every accepted shape.
  * The first call on each device looks up the array's device address
  * (cudaGetSymbolAddress) with that device current; make that first call
  * before any stream capture.  Every call shares the one array and leaves its
- * contents behind (the call clears what must start at zero), so calls that
- * overlap on the GPU -- several streams, or several host threads on one
- * device -- race and must be serialised by the caller.  Device-side checks of
- * this path have no error word the caller can read. */
+ * contents behind: each call first clears the arrival words it uses (one
+ * cudaMemsetAsync on `stream`), so calls that overlap on the GPU --
+ * several streams, or several host threads on one device -- race and must be
+ * serialised by the caller.  The device error word is not cleared by a call:
+ * it keeps the first device error (codes as for grinqh_decode_gemv) until
+ * grinqh_noalloc_check_device_error reads it. */
 int grinqh_decode_gemv_noalloc(const uint32_t *planes, const uint16_t *s, const uint16_t *z,
                                const uint16_t *x, const float *theta, const float *phi,
                                int d_in, int d_out, int b_max, float *y, void *stream);
+
+/* Reads the no-allocation path's device error word on the current device
+ * (synchronises `stream`).  Returns GRINQH_OK, or GRINQH_ERR_DEVICE with the
+ * code in grinqh_last_error(); in that case it also clears the word and the
+ * split-K state a failed call may have left. */
+int grinqh_noalloc_check_device_error(void *stream);
+
+/* Device address and size in bytes of the no-allocation path's fixed array on
+ * the current device, for inspection and tests (the library owns its
+ * contents: the error word is the first int). */
+int grinqh_noalloc_scratch(void **ptr, size_t *bytes);
 
 #ifdef __cplusplus
 }

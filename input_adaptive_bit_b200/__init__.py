@@ -21,6 +21,8 @@ __all__ = [
     "grinqh_gemv_dense4", "grinqh_decode_gemv", "grinqh_decode_gemv_noalloc",
     "grinqh_group_workspace_bytes", "grinqh_decode_gemv_group", "GrinqhLinearDesc", "MAX_GROUP",
     "grinqh_prefill_workspace_bytes", "grinqh_prefill_gemm",
+    "grinqh_noalloc_check_device_error", "grinqh_noalloc_scratch",
+    "grinqh_batch_workspace_bytes", "grinqh_decode_gemv_batch", "MAX_BATCH",
     "EXPORTS",
 ]
 
@@ -35,6 +37,7 @@ ERR_CUDA = -4
 ERR_DEVICE = -5
 
 MAX_GROUP = 4  # GRINQH_MAX_GROUP
+MAX_BATCH = 8  # GRINQH_MAX_BATCH
 
 
 class GrinqhLinearDesc(ctypes.Structure):
@@ -62,6 +65,11 @@ EXPORTS = {
     "grinqh_decode_gemv": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _P, _P, _P, _P, _P, _P,
                                 _Z, _P]),
     "grinqh_decode_gemv_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _P, _P]),
+    "grinqh_noalloc_check_device_error": (_I, [_P]),
+    "grinqh_noalloc_scratch": (_I, [_P, _P]),
+    "grinqh_batch_workspace_bytes": (_Z, []),
+    "grinqh_decode_gemv_batch": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _Z,
+                                      _P]),
     "grinqh_group_workspace_bytes": (_Z, []),
     "grinqh_decode_gemv_group": (_I, [_I, _P, _P, _Z, _P]),
     "grinqh_prefill_workspace_bytes": (_Z, []),
@@ -181,6 +189,33 @@ def grinqh_decode_gemv_noalloc(planes, s, z, x, theta, phi, d_in, d_out, b_max, 
     _check(lib().grinqh_decode_gemv_noalloc(_ptr(planes), _ptr(s), _ptr(z), _ptr(x), _ptr(theta),
                                             _ptr(phi), d_in, d_out, b_max, _ptr(y),
                                             _stream(stream)))
+
+
+def grinqh_noalloc_check_device_error(stream=None):
+    """Raises GrinqhError (status ERR_DEVICE) if a no-allocation call recorded a
+    device error since the last check; clears it."""
+    _check(lib().grinqh_noalloc_check_device_error(_stream(stream)))
+
+
+def grinqh_noalloc_scratch():
+    """(device address, bytes) of the no-allocation path's fixed array on the
+    current device (inspection and tests)."""
+    ptr, nbytes = ctypes.c_void_p(), ctypes.c_size_t()
+    _check(lib().grinqh_noalloc_scratch(ctypes.byref(ptr), ctypes.byref(nbytes)))
+    return int(ptr.value or 0), int(nbytes.value)
+
+
+def grinqh_batch_workspace_bytes() -> int:
+    return lib().grinqh_batch_workspace_bytes()
+
+
+def grinqh_decode_gemv_batch(planes, s, z, x, theta, phi, B, d_in, d_out, b_max, y, u, ws,
+                             ws_bytes, stream=None):
+    """B <= 8 tokens (x fp16 [B][d_in]) through one linear, each with its own widths;
+    y fp32 [B][d_out]; u (uint8 [d_in] union widths) may be None."""
+    _check(lib().grinqh_decode_gemv_batch(_ptr(planes), _ptr(s), _ptr(z), _ptr(x), _ptr(theta),
+                                          _ptr(phi), B, d_in, d_out, b_max, _ptr(y), _ptr(u),
+                                          _ptr(ws), ws_bytes, _stream(stream)))
 
 
 def grinqh_group_workspace_bytes() -> int:

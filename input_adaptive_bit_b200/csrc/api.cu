@@ -75,6 +75,30 @@ int record_error(int code, const char *fmt, ...) {
   return code;
 }
 
+int check_decode_args(const uint32_t *planes, const uint16_t *s, const uint16_t *z,
+                      const uint16_t *x, const float *theta, const float *phi, int d_in, int d_out,
+                      int b_max, const float *y, const int32_t *lists, const int32_t *counts,
+                      const float *grp_sums, const char *who) {
+  TRY(check_bmax(b_max));
+  TRY(check_din(d_in));
+  TRY(check_dout(d_out));
+  if (d_in > kDecodeMaxDin)
+    return fail(GRINQH_ERR_UNSUPPORTED_SHAPE,
+                "%s: d_in must be <= %d (got %d); use grinqh_assign + grinqh_gemv", who,
+                kDecodeMaxDin, d_in);
+  TRY(check_ptr(planes, (d_out / 16) % 4 == 0 ? 16 : 4, "planes"));
+  TRY(check_ptr(s, 16, "s"));
+  TRY(check_ptr(z, 16, "z"));
+  TRY(check_ptr(x, 16, "x"));
+  TRY(check_ptr(theta, 4, "theta"));
+  if (phi) TRY(check_ptr(phi, 4, "phi"));
+  TRY(check_ptr(y, 4, "y"));
+  if (lists) TRY(check_ptr(lists, 4, "lists"));
+  if (counts) TRY(check_ptr(counts, 4, "counts"));
+  if (grp_sums) TRY(check_ptr(grp_sums, 4, "grp_sums"));
+  return GRINQH_OK;
+}
+
 cudaError_t ensure_smem_attr(const void *kernel, size_t bytes) {
   // One bit per (device, kernel slot); a handful of kernels use this.
   static std::atomic<unsigned long long> done[64];
@@ -181,24 +205,8 @@ int grinqh_decode_gemv(const uint32_t *planes, const uint16_t *s, const uint16_t
                        int d_out, int b_max, float *y, uint8_t *b, int32_t *lists,
                        int32_t *counts, float *grp_sums, void *ws, size_t ws_bytes,
                        void *stream) {
-  TRY(check_bmax(b_max));
-  TRY(check_din(d_in));
-  TRY(check_dout(d_out));
-  if (d_in > grinqh::kDecodeMaxDin)
-    return fail(GRINQH_ERR_UNSUPPORTED_SHAPE,
-                "grinqh_decode_gemv: d_in must be <= %d (got %d); use grinqh_assign + "
-                "grinqh_gemv",
-                grinqh::kDecodeMaxDin, d_in);
-  TRY(check_ptr(planes, (d_out / 16) % 4 == 0 ? 16 : 4, "planes"));
-  TRY(check_ptr(s, 16, "s"));
-  TRY(check_ptr(z, 16, "z"));
-  TRY(check_ptr(x, 16, "x"));
-  TRY(check_ptr(theta, 4, "theta"));
-  if (phi) TRY(check_ptr(phi, 4, "phi"));
-  TRY(check_ptr(y, 4, "y"));
-  if (lists) TRY(check_ptr(lists, 4, "lists"));
-  if (counts) TRY(check_ptr(counts, 4, "counts"));
-  if (grp_sums) TRY(check_ptr(grp_sums, 4, "grp_sums"));
+  TRY(grinqh::check_decode_args(planes, s, z, x, theta, phi, d_in, d_out, b_max, y, lists, counts,
+                                grp_sums, "grinqh_decode_gemv"));
   TRY(check_ptr(ws, 256, "ws"));
   const size_t need = grinqh::ws_layout(d_in, d_out, b_max).total;
   if (ws_bytes < need)
@@ -208,6 +216,26 @@ int grinqh_decode_gemv(const uint32_t *planes, const uint16_t *s, const uint16_t
                                            b, lists, counts, grp_sums, ws,
                                            (cudaStream_t)stream),
                      "grinqh_decode_gemv launch");
+}
+
+size_t grinqh_batch_workspace_bytes(void) { return grinqh::batch_ws_bytes(); }
+
+int grinqh_decode_gemv_batch(const uint32_t *planes, const uint16_t *s, const uint16_t *z,
+                             const uint16_t *x, const float *theta, const float *phi, int B,
+                             int d_in, int d_out, int b_max, float *y, uint8_t *u, void *ws,
+                             size_t ws_bytes, void *stream) {
+  if (B < 1 || B > GRINQH_MAX_BATCH)
+    return fail(GRINQH_ERR_INVALID_ARG, "grinqh_decode_gemv_batch: B must be in [1, %d] (got %d)",
+                GRINQH_MAX_BATCH, B);
+  TRY(grinqh::check_decode_args(planes, s, z, x, theta, phi, d_in, d_out, b_max, y, nullptr,
+                                nullptr, nullptr, "grinqh_decode_gemv_batch"));
+  TRY(check_ptr(ws, 256, "ws"));
+  if (ws_bytes < grinqh::batch_ws_bytes())
+    return fail(GRINQH_ERR_WORKSPACE_TOO_SMALL, "workspace of %zu bytes, batch decode needs %zu",
+                ws_bytes, grinqh::batch_ws_bytes());
+  return cuda_status(grinqh::launch_decode_batch(planes, s, z, x, theta, phi, B, d_in, d_out,
+                                                 b_max, y, u, ws, (cudaStream_t)stream),
+                     "grinqh_decode_gemv_batch launch");
 }
 
 size_t grinqh_prefill_workspace_bytes(void) { return grinqh::prefill_ws_bytes(); }

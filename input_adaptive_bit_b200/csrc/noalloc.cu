@@ -8,9 +8,9 @@
 // synchronise the device).  Such a caller cannot provide the workspace that
 // grinqh_decode_gemv needs.  This entry point runs the fused decode kernel
 // (without its optional outputs) and keeps what is neither an input nor the
-// output -- the split-K partial sums, their arrival counters and the error
-// word -- in one fixed-size array that the library reserves on every GPU that
-// loads it and holds until the process exits.
+// output -- the split-K partial sums, their arrival words and the device
+// error word -- in one fixed-size array that the library reserves
+// on every GPU that loads it and holds until the process exits.
 #include <mutex>
 
 #include "grinqh_internal.cuh"
@@ -18,19 +18,17 @@
 namespace grinqh {
 namespace {
 
-constexpr int kNoAllocMaxDin = 32768;   // largest d_in this entry point accepts
-constexpr int kNoAllocMaxDout = 32768;  // largest d_out
+// Scratch layout: the error word (a 256-byte header), the split-K arrival
+// words (64-bit, two per 1024-output tile: enough for d_out up to 2^24), then
+// the partial sums of up to kMaxCtas CTAs.  None of it depends on d_in, so the
+// scratch serves every shape grinqh_decode_gemv takes.
+constexpr size_t kNaCounters = 256;
+constexpr size_t kNaPartials = kNaCounters + (size_t)2 * ((1 << 24) / 1024) * 8;
+constexpr size_t kNoAllocBytes = kNaPartials + (size_t)kMaxCtas * 1024 * 4;  // about 1.2 MB
+static_assert(kNaPartials % 256 == 0, "aligned regions");
 
-constexpr size_t a256(size_t v) { return (v + 255) & ~size_t(255); }
-// The workspace layout of grinqh_workspace_bytes at the largest accepted shape
-// (header, counters, the two-call path's unit stream, partial sums).
-constexpr size_t kNoAllocBytes =
-    a256(a256(a256(a256(sizeof(WsHeader) + (size_t)kMaxTiles * 4) + (size_t)kNoAllocMaxDin * 16) +
-              (size_t)kNoAllocMaxDin * 16) +
-         (size_t)kMaxCtas * 2 * kTileOut * 4);
-
-// The scratch (about 2.2 MB).  In host code this name is only a host-side
-// stand-in; kernels get the device address from cudaGetSymbolAddress.
+// The scratch.  In host code this name is only a host-side stand-in; kernels
+// get the device address from cudaGetSymbolAddress.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
 
 std::mutex g_mu;
@@ -62,28 +60,69 @@ extern "C" int grinqh_decode_gemv_noalloc(const uint32_t *planes, const uint16_t
                                           const float *theta, const float *phi, int d_in,
                                           int d_out, int b_max, float *y, void *stream) {
   using namespace grinqh;
-  if (grinqh_workspace_bytes(d_in, d_out, b_max) == 0)
-    return GRINQH_ERR_UNSUPPORTED_SHAPE;  // message set by the shape check
-  if (d_in > kNoAllocMaxDin || d_out > kNoAllocMaxDout)
-    return record_error(GRINQH_ERR_UNSUPPORTED_SHAPE,
-                        "grinqh_decode_gemv_noalloc: d_in and d_out must be <= 32768 (its fixed "
-                        "scratch); got d_in=%d d_out=%d",
-                        d_in, d_out);
+  // every check first: nothing is queued on a failed call
+  const int rc = check_decode_args(planes, s, z, x, theta, phi, d_in, d_out, b_max, y, nullptr,
+                                   nullptr, nullptr, "grinqh_decode_gemv_noalloc");
+  if (rc != GRINQH_OK) return rc;
   void *base = nullptr;
   cudaError_t e = scratch_address(&base);
   if (e != cudaSuccess)
     return record_error(GRINQH_ERR_CUDA, "grinqh_decode_gemv_noalloc: scratch address: %s",
                         cudaGetErrorString(e));
   char *sc = static_cast<char *>(base);
-  // Every call shares the array, which keeps the last call's contents.  The
-  // kernel leaves its counters at zero, but the error word and the counters of a
-  // call that gave up would stay set: they are cleared first.  (The clear also
-  // keeps the kernel from overlapping the kernel before it on the stream.)
-  const WsLayout L = ws_layout(d_in, d_out, b_max);
-  e = cudaMemsetAsync(sc, 0, L.counters + (size_t)L.tiles * 4, (cudaStream_t)stream);
+  // Every call shares the array, which keeps the last call's contents.  A
+  // completed call leaves its arrival words at zero, but one that gave up would
+  // not: the words this shape uses are cleared first.  The error word is not:
+  // it keeps the first error until it is read.
+  const size_t tiles = ((size_t)d_out + 1023) / 1024;
+  e = cudaMemsetAsync(sc + kNaCounters, 0, 2 * tiles * 8 > 148 * 8 ? 2 * tiles * 8 : 148 * 8,
+                      (cudaStream_t)stream);
   if (e != cudaSuccess)
     return record_error(GRINQH_ERR_CUDA, "grinqh_decode_gemv_noalloc: clearing scratch: %s",
                         cudaGetErrorString(e));
-  return grinqh_decode_gemv(planes, s, z, x, theta, phi, d_in, d_out, b_max, y, nullptr, nullptr,
-                            nullptr, nullptr, sc, kNoAllocBytes, stream);
+  e = launch_decode_split(planes, s, z, x, theta, phi, d_in, d_out, b_max, y, nullptr, nullptr,
+                          nullptr, nullptr, reinterpret_cast<unsigned long long *>(sc + kNaCounters),
+                          reinterpret_cast<float *>(sc + kNaPartials), reinterpret_cast<int *>(sc),
+                          (cudaStream_t)stream);
+  if (e != cudaSuccess)
+    return record_error(GRINQH_ERR_CUDA, "grinqh_decode_gemv_noalloc launch: %s",
+                        cudaGetErrorString(e));
+  return record_error(GRINQH_OK, "");
+}
+
+extern "C" int grinqh_noalloc_check_device_error(void *stream) {
+  using namespace grinqh;
+  void *base = nullptr;
+  cudaError_t e = scratch_address(&base);
+  if (e != cudaSuccess)
+    return record_error(GRINQH_ERR_CUDA, "grinqh_noalloc_check_device_error: scratch address: %s",
+                        cudaGetErrorString(e));
+  cudaStream_t st = (cudaStream_t)stream;
+  int code = 0;
+  e = cudaMemcpyAsync(&code, base, sizeof code, cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e == cudaSuccess && code != 0) {
+    // clear the error word and the split-K state a failed call may have left
+    e = cudaMemsetAsync(base, 0, kNaPartials, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  }
+  if (e != cudaSuccess)
+    return record_error(GRINQH_ERR_CUDA, "grinqh_noalloc_check_device_error: %s",
+                        cudaGetErrorString(e));
+  if (code != 0) return record_error(GRINQH_ERR_DEVICE, "device error code %d", code);
+  return record_error(GRINQH_OK, "");
+}
+
+extern "C" int grinqh_noalloc_scratch(void **ptr, size_t *bytes) {
+  using namespace grinqh;
+  if (ptr == nullptr || bytes == nullptr)
+    return record_error(GRINQH_ERR_INVALID_ARG, "grinqh_noalloc_scratch: ptr and bytes must not be NULL");
+  void *base = nullptr;
+  cudaError_t e = scratch_address(&base);
+  if (e != cudaSuccess)
+    return record_error(GRINQH_ERR_CUDA, "grinqh_noalloc_scratch: scratch address: %s",
+                        cudaGetErrorString(e));
+  *ptr = base;
+  *bytes = kNoAllocBytes;
+  return record_error(GRINQH_OK, "");
 }

@@ -237,7 +237,7 @@ def test_uniform_sweep_llama_up_proj(idx, path):
 
 
 @pytest.mark.slow
-@pytest.mark.parametrize("idx", [0, 1, 3, 5])
+@pytest.mark.parametrize("idx", range(len(synth.config3())))
 @pytest.mark.parametrize("path", PATHS)
 def test_70b_shapes_redrawn_inputs(idx, path):
     spec = synth.config3()[idx]
@@ -253,8 +253,13 @@ def test_70b_shapes_redrawn_inputs(idx, path):
 
 
 @pytest.mark.slow
+@pytest.mark.parametrize("layer", [0, 31])
 @pytest.mark.parametrize("path", PATHS)
-def test_llama3_8b_layer_of_the_decode_step(path):
-    for spec in synth.config4(n_layers=1):
+def test_llama3_8b_layers_of_the_decode_step(layer, path):
+    # all 7 linears (q, k, v, o, gate, up, down) of the first and the last of the
+    # 32 layers of the decode step, each with its own weights, x and theta
+    specs = [s for s in synth.config4() if s.name.startswith(f"L{layer}.")]
+    assert len(specs) == 7
+    for spec in specs:
         case = synth.make_case(spec)
         full_case_check(case, sample_outputs=128, sample_rows=32, path=path)
