@@ -525,6 +525,20 @@ def uniform_sweep_fit(device, reps=20):
         d4(x, y=y, stream=st)
 
     us_d4 = (_graph_ms(torch, st, dense, reps) / reps - t_flush) * 1e3
+    # the same 4 bits per weight on the product's own machinery: a 4-bit base (b_max 4)
+    # with every row read at full width is a dense 4-bit GEMV in the plane layout
+    q4p, s4p, z4p = synth.rtn_quantize(
+        synth.gaussian_weights(synth.rng(spec.config_id, spec.layer, 0), spec.d_in, spec.d_out), 4)
+    lin4 = GrinqhLinear(q4p, s4p, z4p, 4, device=device)
+    del q4p
+    th4 = torch.from_numpy(synth.uniform_thresholds(4, 4)).to(device)
+
+    def dense_same():
+        flush()
+        lin4.decode(x, th4, y=y, outputs=False, stream=st)
+
+    us_d4s = (_graph_ms(torch, st, dense_same, reps) / reps - t_flush) * 1e3
+    del lin4
     bits = np.array([p[0] for p in pts], np.float64)
     t = np.array([p[1] for p in pts], np.float64)
     c, a = np.polyfit(bits, t, 1)
@@ -537,7 +551,13 @@ def uniform_sweep_fit(device, reps=20):
             "points": [{"bits": b, "us": round(u, 2), "GBps": round(n / (u * 1e3), 1)}
                        for b, u, n in pts],
             "dense4_us": round(us_d4, 2), "dense4_GBps": round(d4_bytes / (us_d4 * 1e3), 1),
-            "time_4bit_vs_dense4": round(pts[1][1] / us_d4, 3)}
+            "time_4bit_vs_dense4": round(pts[1][1] / us_d4, 3),
+            "dense4_same_kernel_us": round(us_d4s, 2),
+            "dense4_same_kernel_GBps": round(d4_bytes / (us_d4s * 1e3), 1),
+            "time_4bit_vs_dense4_same_kernel": round(pts[1][1] / us_d4s, 3),
+            "dense4_how": "dense4: grinqh_gemv_dense4 (nibble layout, its own kernel); "
+                          "dense4_same_kernel: grinqh_decode_gemv on a 4-bit base with every row "
+                          "at width 4 (the same bytes, the product's kernel)"}
 
 
 def seventy_b_pair(device, peak, n_pool=64, reps=4):

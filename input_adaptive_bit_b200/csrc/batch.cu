@@ -21,11 +21,11 @@
 //    group's s and adds them into its outputs when the group of the half stage
 //    it starts changes.  The group
 //    terms s Phi_{g,t} + z X_{g,t} (per token) are added once per window.
-//  * Copies, mbarrier ring and split-K are those of the batch-1 kernel: four copy
-//    warps stream 256-byte segments with 16-byte cp.async copies, eight MMA warps (one per
-//    128-output block) decode them, and the partial tiles of a tile's CTAs meet first in cluster pairs
-//    through distributed shared memory, then in global memory, where the last
-//    arrival sums them in a fixed order (y is deterministic).
+//  * Copies, mbarrier ring and split-K follow the batch-1 kernel: four copy warps
+//    stream 256-byte segments with 16-byte cp.async copies, eight MMA warps (one
+//    per 128-output block) decode them, and the partial tiles of a tile's CTAs
+//    meet in global memory, where the last arrival sums them in a fixed order
+//    (y is deterministic).
 #include "grinqh_internal.cuh"
 #include "pipeline.cuh"
 
@@ -53,7 +53,8 @@ constexpr int kRound = 1024;                    // units per round
 constexpr int kSlots = 8;                       // groups per window
 constexpr int kChunkRows = 32;
 constexpr int kPolls = 1 << 20;                 // bounded poll for a missing split-K partial
-constexpr int kGrpPad = 2 * kK;                 // a group's units are padded to this: a warp's half stage
+constexpr int kGrpPad = 2 * kK;
+constexpr int kFixParts = 32;                   // partial tiles staged per pass of the split-K sum                 // a group's units are padded to this: a warp's half stage
 
 // workspace: header, 64-bit arrival words, partial tiles [CTA][kNB][kTile]
 constexpr size_t kWsCounters = sizeof(WsHeader);
@@ -97,7 +98,7 @@ struct BatchArgs {
   const uint16_t *x;   // [B][d_in]
   const float *theta;
   const float *phi;    // may be null: the default table
-  int B, d_in, d_out, b_max, P, W, G, tiles, m, cl;
+  int B, d_in, d_out, b_max, P, W, G, tiles, m;
   float *y;            // [B][d_out]
   uint8_t *u;          // optional [d_in]: union widths (null: not written)
   unsigned long long *counters;
@@ -170,7 +171,7 @@ __global__ void __launch_bounds__(kThreads, 1) batch_kernel(const __grid_constan
   asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
   __half2 t2[4];
   sort_thresholds(th_raw, t2);
-  if (c >= C_eff) return;  // (whole clusters: the host makes C_eff a multiple of the cluster size)
+  if (c >= C_eff) return;
   __syncthreads();
 
   uint64_t policy = 0;
@@ -553,39 +554,10 @@ __global__ void __launch_bounds__(kThreads, 1) batch_kernel(const __grid_constan
     }
     __syncthreads();
 
-    // ---- split-K (as in decode.cu), B tokens x the share's outputs ----
-    int cl_n = 1, rank = 0;
-    if (a.cl) {
-      asm("mov.u32 %0, %%cluster_nctarank;" : "=r"(cl_n));
-      rank = (int)cluster_rank();
-    }
-    const int nsh = m == 1 ? kTile : kTile / cl_n, sh0 = m == 1 ? 0 : rank * nsh;
-    const int nq = B * (nsh / 4);  // float4s of the share
-    if (a.cl && m > 1) {
-      cluster_arrive();
-      cluster_wait();
-      for (int q = tid; q < nq; q += kThreads) {
-        const int t = q / (nsh / 4), o4 = q % (nsh / 4);
-        float4 v = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-        for (int k = 0; k < cl_n; ++k) v = f4add(v, ld_peer_f4(s_part + t * kTile + sh0 + 4 * o4, (uint32_t)k));
-        // the cluster sum goes to this CTA's own s_part slot of the share only after
-        // every peer has read it: written to global (or y) directly instead
-        if (m == cl_n) {
-          const int o = obase + sh0 + 4 * o4;
-          if (o < a.d_out) {
-            float *yo = a.y + (size_t)t * a.d_out + o;
-            yo[0] = v.x;
-            yo[1] = v.y;
-            yo[2] = v.z;
-            yo[3] = v.w;
-          }
-        } else {
-          reinterpret_cast<float4 *>(a.partials + ((size_t)c * kNB + t) * kTile + sh0)[o4] = v;
-        }
-      }
-      cluster_arrive();
-    } else if (m == 1) {
-      for (int q = tid; q < nq; q += kThreads) {
+    // ---- split-K (as in decode.cu): publish, count the arrival; the last arrival sums
+    // the m partials of every token in CTA order, staging them in shared memory ----
+    if (m == 1) {
+      for (int q = tid; q < B * (kTile / 4); q += kThreads) {
         const int t = q / (kTile / 4), o4 = q % (kTile / 4);
         const float4 v = reinterpret_cast<const float4 *>(s_part + t * kTile)[o4];
         const int o = obase + 4 * o4;
@@ -597,91 +569,65 @@ __global__ void __launch_bounds__(kThreads, 1) batch_kernel(const __grid_constan
           yo[3] = v.w;
         }
       }
-    } else {
-      for (int q = tid; q < nq; q += kThreads) {
-        const int t = q / (kTile / 4), o4 = q % (kTile / 4);
-        reinterpret_cast<float4 *>(a.partials + ((size_t)c * kNB + t) * kTile)[o4] =
-            reinterpret_cast<const float4 *>(s_part + t * kTile)[o4];
+      continue;
+    }
+    const int c_first = (c / m) * m;
+    for (int q = tid; q < B * (kTile / 4); q += kThreads) {
+      const int t = q / (kTile / 4), o4 = q % (kTile / 4);
+      reinterpret_cast<float4 *>(a.partials + ((size_t)c * kNB + t) * kTile)[o4] =
+          reinterpret_cast<const float4 *>(s_part + t * kTile)[o4];
+    }
+    __syncthreads();
+    if (tid == 0) {
+      unsigned long long *word = a.counters + tile;
+      const bool masked = m <= 32;
+      const unsigned fullm = !masked ? 0u : m == 32 ? 0xffffffffu : (1u << m) - 1u;
+      const unsigned long long add = (1ull << 32) | (masked ? 1ull << part : 0ull);
+      asm volatile("fence.acq_rel.gpu;\n" ::: "memory");
+      const unsigned long long old = atomicAdd(word, add);
+      const bool last = (unsigned)(old >> 32) == (unsigned)(m - 1);
+      if (last) {
+        if (masked && (((unsigned)old | (unsigned)add) & fullm) != fullm) {
+          int polls = 0;
+          while ((unsigned)(ld_acquire64(word) & fullm) != fullm && ++polls < kPolls) __nanosleep(64);
+          atomicCAS(a.error, 0, kDevErrSplitKTimeout);
+        }
+        asm volatile("fence.acq_rel.gpu;\n" ::: "memory");
+        *reinterpret_cast<volatile unsigned long long *>(word) = 0ull;
+      }
+      s_misc[1] = last ? 1 : 0;
+    }
+    __syncthreads();
+    if (s_misc[1]) {
+      float4 *stage = reinterpret_cast<float4 *>(smem);  // [kFixParts][kTile / 4], the idle ring
+      for (int t = 0; t < B; ++t) {
+        float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        for (int k0 = 0; k0 < m; k0 += kFixParts) {
+          const int np = min(kFixParts, m - k0);
+          for (int q = tid; q < np * (kTile / 4); q += kThreads) {
+            const int k = q / (kTile / 4), o4 = q % (kTile / 4);
+            cp_async16(stage + q, a.partials + ((size_t)(c_first + k0 + k) * kNB + t) * kTile + 4 * o4, 16);
+          }
+          cp_async_commit();
+          cp_async_wait<0>();
+          __syncthreads();
+          if (tid < kTile / 4)
+            for (int k = 0; k < np; ++k) acc = f4add(acc, stage[k * (kTile / 4) + tid]);
+          __syncthreads();
+        }
+        const int o = obase + 4 * tid;
+        if (tid < kTile / 4 && o < a.d_out) {
+          float *yo = a.y + (size_t)t * a.d_out + o;
+          yo[0] = acc.x;
+          yo[1] = acc.y;
+          yo[2] = acc.z;
+          yo[3] = acc.w;
+        }
       }
     }
-    const int npart = m / cl_n;
-    if (m > 1 && npart > 1) {
-      const int c_first = (c / m) * m, kidx = (c - c_first) / cl_n;
-      __syncthreads();
-      if (tid == 0) {
-        unsigned long long *word = a.counters + (a.cl ? tile * cl_n + rank : tile);
-        const bool masked = npart <= 32;
-        const unsigned fullm = !masked ? 0u : npart == 32 ? 0xffffffffu : (1u << npart) - 1u;
-        const unsigned long long add = (1ull << 32) | (masked ? 1ull << kidx : 0ull);
-        __threadfence();
-        const unsigned long long old = atomicAdd(word, add);
-        const bool last = (unsigned)(old >> 32) == (unsigned)(npart - 1);
-        if (last) {
-          if (masked && (((unsigned)old | (unsigned)add) & fullm) != fullm) {
-            int polls = 0;
-            while ((unsigned)(ld_acquire64(word) & fullm) != fullm && ++polls < kPolls) __nanosleep(64);
-            atomicCAS(a.error, 0, kDevErrSplitKTimeout);
-          }
-          __threadfence();
-          *reinterpret_cast<volatile unsigned long long *>(word) = 0ull;
-        }
-        s_misc[1] = last ? 1 : 0;
-      }
-      __syncthreads();
-      if (s_misc[1]) {
-        for (int q = tid; q < nq; q += kThreads) {
-          const int t = q / (nsh / 4), o4 = q % (nsh / 4);
-          float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-          for (int k = 0; k < npart; ++k)
-            acc = f4add(acc, __ldcg(reinterpret_cast<const float4 *>(
-                                        a.partials + ((size_t)(c_first + k * cl_n + rank) * kNB + t) * kTile +
-                                        sh0) +
-                                    o4));
-          const int o = obase + sh0 + 4 * o4;
-          if (o < a.d_out) {
-            float *yo = a.y + (size_t)t * a.d_out + o;
-            yo[0] = acc.x;
-            yo[1] = acc.y;
-            yo[2] = acc.z;
-            yo[3] = acc.w;
-          }
-        }
-      }
-    }
-    if (a.cl && m > 1) cluster_wait();
   }
   if (warp == kMmaWarps && sz_phase > 0) ok &= mbar_wait(sz_bar, (sz_phase - 1) & 1u, a.error);
   (void)ok;
-}
-
-template <bool ALIGNED>
-int cluster_capacity(int cl) {
-  static int cached[64][3] = {{0}};
-  const int idx = cl == 2 ? 1 : cl == 4 ? 2 : 0;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return 0;
-  if (cached[dev][idx]) return cached[dev][idx] - 1;
-  int n = 0;
-  if (ensure_smem_attr((const void *)batch_kernel<ALIGNED>, kSmBytes) == cudaSuccess) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(cl * 4);
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = kSmBytes;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = cl;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    int clusters = 0;
-    if (cudaOccupancyMaxActiveClusters(&clusters, batch_kernel<ALIGNED>, &cfg) == cudaSuccess)
-      n = clusters * cl;
-    else
-      (void)cudaGetLastError();
-  }
-  cached[dev][idx] = n + 1;
-  return n;
 }
 
 int device_sms() {
@@ -692,7 +638,7 @@ int device_sms() {
 }
 
 template <bool ALIGNED>
-cudaError_t launch(const BatchArgs &a, int C, int cl, cudaStream_t st) {
+cudaError_t launch(const BatchArgs &a, int C, cudaStream_t st) {
   cudaError_t e = ensure_smem_attr((const void *)batch_kernel<ALIGNED>, kSmBytes);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -700,15 +646,11 @@ cudaError_t launch(const BatchArgs &a, int C, int cl, cudaStream_t st) {
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = kSmBytes;
   cfg.stream = st;
-  cudaLaunchAttribute attr[2];
+  cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
-  attr[1].id = cudaLaunchAttributeClusterDimension;
-  attr[1].val.clusterDim.x = cl;
-  attr[1].val.clusterDim.y = 1;
-  attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = cl > 1 ? 2 : 1;
+  cfg.numAttrs = 1;
   e = cudaLaunchKernelEx(&cfg, batch_kernel<ALIGNED>, a);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
@@ -746,13 +688,7 @@ cudaError_t launch_decode_batch(const uint32_t *planes, const uint16_t *s, const
   const bool aligned = a.W % 4 == 0;
   const int C = device_sms();
   a.m = a.tiles >= C ? 1 : C / a.tiles;
-  // cluster pairs where the tile's CTAs pair up and the device holds every pair at once
-  int cl = 1;
-  if (a.m > 1 && a.m % 2 == 0 && C % 2 == 0 &&
-      (aligned ? cluster_capacity<true>(2) : cluster_capacity<false>(2)) >= C)
-    cl = 2;
-  a.cl = cl > 1 ? 1 : 0;
-  return aligned ? launch<true>(a, C, cl, st) : launch<false>(a, C, cl, st);
+  return aligned ? launch<true>(a, C, st) : launch<false>(a, C, st);
 }
 
 }  // namespace grinqh

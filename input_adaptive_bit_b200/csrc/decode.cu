@@ -15,18 +15,21 @@
 //    2-bit field of plane p.  X_g, Phi_g are per-group sums of x and x phi.
 //  * Work = 1024-output tiles x row slices.  A unit's tile segment is 256
 //    contiguous bytes of its plane region.  Each tile's d_in rows are cut into
-//    m contiguous slices, one per CTA (one wave); every CTA derives its own
-//    units from x and theta -- one row per lane, a ballot per plane, a scan of
-//    the per-(group, plane, 32-row chunk) counts -- so no other kernel and no
-//    global round trip sit between x and the GEMV.  Units are ordered by
-//    group, plane, row.
-//  * Warp roles.  Four copy warps stream the units' segments into an 8-stage
-//    shared-memory ring with 16-byte cp.async copies (L2 evict-first: the planes
-//    are read once), each stage completing on its own "full" mbarrier;
-//    sixteen MMA warps wait on "full", decode, and release the stage on its
-//    "empty" mbarrier.  No block-wide barrier sits inside the loop, so the
-//    MMA warps drift apart and the integer (field extraction) and tensor
-//    (MMA) phases of different warps overlap.
+//    m = floor(CTAs / tiles) contiguous slices, one per CTA (one wave); every
+//    CTA derives its own units from x and theta -- one row per lane, a ballot
+//    per plane, a scan of the per-(group, plane, 32-row chunk) counts -- so no
+//    other kernel and no global round trip sit between x and the GEMV.  Units
+//    are ordered by group, plane, row.
+//  * The m partial tiles of a tile meet in global memory: every CTA of the tile
+//    publishes its partial, waits until all m have arrived, and adds up its own
+//    1/m share of the outputs over the m partials in CTA order (deterministic).
+//    A CTA that waits too long (another CTA of the tile is not running: the GPU
+//    is shared) marks the tile's arrival word and exits; the tile's last
+//    arrival sees the mark and sums the whole tile, so y never depends on the
+//    CTAs being resident together.
+//  * A CTA walks its range in windows of 8 groups and rounds of at most 2048
+//    units.  The segments stream through an 8-stage shared-memory ring
+//    (cp.async, 16 B per thread and copy, one barrier per 64-unit stage).
 //  * The contraction runs on the tensor cores as m16n8k16 MMAs with fp32
 //    accumulation: A (16 outputs x 16 units) is built in registers straight
 //    from the packed words -- a byte permute pairs the same 16 outputs of two
@@ -35,19 +38,10 @@
 //    (16 units x 8) holds x 4^(P-1-p) 2^-c_g in the column of the unit's group
 //    slot j in the window (2 (j mod 4) + j / 4), so the 8 columns keep the
 //    window's 8 groups apart and the group scales s are applied once per
-//    round, not per unit.  One warp covers 128 outputs with 8 MMAs per 16
-//    units: 4 shared loads, 4 permutes, 4 shifts, 32 ANDs and 8 MMAs per 512
-//    bytes of planes.
-//  * Split-K without waiting on other CTAs.  The m partial tiles of a tile
-//    are added in a fixed order (deterministic y).  Where the tile's CTAs form
-//    thread-block clusters of CL (the hardware runs a cluster's CTAs at the
-//    same time), each cluster first adds its CL partials through distributed
-//    shared memory, CTA r of the cluster taking the r-th 1/CL of the outputs;
-//    the m/CL cluster sums of each such share (or the m partials, without
-//    clusters) then meet in global memory, where the last CTA to arrive on
-//    the share's arrival word adds them up.  No CTA ever waits for a CTA
-//    outside its cluster, so the result does not depend on which CTAs are
-//    resident.
+//    round, not per unit.  One warp covers 128 outputs with
+//    8 MMAs per 16 units: 4 shared loads, 4 permutes, 4 shifts, 32 ANDs and
+//    8 MMAs per 512 bytes of planes, against about 240 instructions for a
+//    scalar fp32 decode of the same bytes.
 #include "grinqh_internal.cuh"
 #include "pipeline.cuh"
 
@@ -56,31 +50,31 @@ namespace {
 
 using namespace pipe;
 
-constexpr int kMmaWarps = 16;                   // warps that decode and run the MMAs
-constexpr int kMmaThreads = kMmaWarps * 32;
-constexpr int kCopyWarps = 4;                   // warps that stream the planes into the ring
-constexpr int kCopyThreads = kCopyWarps * 32;
-constexpr int kThreads = kMmaThreads + kCopyThreads;
-constexpr int kBlocks = 8;                      // 128-output blocks of a tile; warps w and w + 8 share one
-constexpr int kTile = 1024;                     // outputs per CTA tile (8 blocks x 128)
-constexpr int kTileW = kTile / 16;              // 64 words = 256 bytes per unit and tile
-constexpr int kRow = kTileW + 4;                // shared words per unit row: conflict-free fragment loads
-constexpr int kK = 16;                          // units per MMA k-step
-constexpr int kStage = 64;                      // units per ring stage (4 k-steps, 2 per warp)
-constexpr int kRing = 8;                        // ring stages
-constexpr int kXSlot = 6;                       // first ring slot of the output CTAs' x cache
-constexpr int kRound = 2048;                    // units per round
-constexpr int kSlots = 8;                       // groups per window (the MMA n dimension)
+constexpr int kThreads = 512;
+constexpr int kWarps = kThreads / 32;
+constexpr int kBlocks = 8;            // 128-output blocks of a tile; warps w and w + 8 share one
+constexpr int kTile = 1024;           // outputs per CTA tile (8 blocks x 128)
+constexpr int kTileW = kTile / 16;    // 64 words = 256 bytes per unit and tile
+constexpr int kRow = kTileW + 4;      // shared words per unit row: conflict-free fragment loads
+constexpr int kK = 16;                // units per MMA k-step
+constexpr int kStage = 64;            // units per ring stage (4 k-steps, 2 per warp)
+constexpr int kRing = 8;              // ring stages
+constexpr int kXSlot = 6;             // first ring slot of the output CTAs' x cache
+constexpr int kRound = 2048;          // units per round
+constexpr int kSlots = 8;             // groups per window (the MMA n dimension)
 constexpr int kMaxG = kDecodeMaxDin / kGroup;
-constexpr int kXCache = 16384;                  // rows of x held in shared memory (output CTAs)
-constexpr int kGT = 16;                         // output CTAs: threads per group, one 8-row chunk each
-constexpr int kChunkRows = 32;                  // GEMV front end: rows per warp chunk, one per lane
-constexpr int kOutCtas = 4;                     // CTAs that write the optional outputs
-constexpr int kMaxGroup = GRINQH_MAX_GROUP;     // linears of one grouped launch
-constexpr int kFlagPolls = 1 << 20;             // bounded poll for a missing split-K partial
+constexpr int kXCache = 16384;        // rows of x held in shared memory
+constexpr int kGT = 16;               // output CTAs: threads per group, one 8-row chunk each
+constexpr int kChunkRows = 32;        // GEMV front end: rows per warp chunk, one per lane
+constexpr int kSpinLimit = 1 << 20;   // polls of a split-K arrival word before giving up (~0.3 s)
+constexpr int kFixParts = 40;         // whole partial tiles staged per pass of a full-tile sum
+constexpr unsigned kCountMask = 0xffffu;   // arrival word: the count of arrived CTAs ...
+constexpr unsigned kGaveUp = 1u << 31;     // ... and the mark of a CTA that stopped waiting
+constexpr int kOutCtas = 4;           // CTAs that write the optional outputs
+constexpr int kMaxGroup = GRINQH_MAX_GROUP;  // linears of one grouped launch
 
-// workspace of a grouped launch: the header, the 64-bit arrival words of every
-// linear's split tiles (fixed offset), then the partial tiles of every CTA
+// workspace of a grouped launch: the header, the arrival words of every linear's
+// tiles (fixed offset), then the partial tiles of every CTA
 constexpr size_t kGroupWsCounters = sizeof(WsHeader);
 constexpr size_t kGroupWsPartials = (kGroupWsCounters + (size_t)kMaxTiles * 4 + 255) & ~size_t(255);
 
@@ -95,33 +89,31 @@ constexpr size_t kSmBfrag = kSmUx + kRound * 4;                             // u
 constexpr size_t kSmS = kSmBfrag + (size_t)(kRound / kK) * 32 * 8;          // fp16 [kSlots][kTile]
 constexpr size_t kSmZ = kSmS + (size_t)kSlots * kTile * 2;                  // fp16 [kSlots][kTile]
 constexpr size_t kSmSlot = kSmZ + (size_t)kSlots * kTile * 2;               // SlotInfo [kSlots]
-constexpr size_t kSmRed = kSmSlot + kSlots * 16;                            // fp32 [kTile]: the CTA's partial
+constexpr size_t kSmRed = kSmSlot + kSlots * 16;                            // fp32 [kTile]: odd-k warps
 constexpr size_t kSmChunkCnt = kSmRed + (size_t)kTile * 4;                  // i32 [kSlots][4][4]: units per
                                                                             // (slot, plane, chunk)
-constexpr size_t kSmWarpSum = kSmChunkCnt + kSlots * 4 * 4 * 4;             // float4 [kMmaWarps]: X, Phi, max|x|
-constexpr size_t kSmWarpBal = kSmWarpSum + kMmaWarps * 16;                  // u32 [kMmaWarps][2][4]: ballots
-constexpr size_t kSmWarpOff = kSmWarpBal + kMmaWarps * 32;                  // i32 [kMmaWarps][2][4]: first units
-constexpr size_t kSmBar = kSmWarpOff + kMmaWarps * 32;                      // u64: full[kRing], empty[kRing], sz
-constexpr size_t kSmMisc = kSmBar + (2 * kRing + 1) * 8;                    // i32 [4]: window units, last flag
+constexpr size_t kSmWarpSum = kSmChunkCnt + kSlots * 4 * 4 * 4;             // float4 [kWarps]: X, Phi, max|x|
+constexpr size_t kSmWarpBal = kSmWarpSum + kWarps * 16;                     // u32 [kWarps][2][4]: ballots
+constexpr size_t kSmWarpOff = kSmWarpBal + kWarps * 32;                     // i32 [kWarps][2][4]: first units
+constexpr size_t kSmMisc = kSmWarpOff + kWarps * 32;                        // i32 [4]: the last-arrival flag
 constexpr size_t kSmBytes = kSmMisc + 16;
 // the output CTAs keep their counts and scans where the GEMV CTAs have the ring
 constexpr size_t kSmCnt = kSmRing;                                          // u32 [kMaxG]: plane counts, bytes
 constexpr size_t kSmLoff = kSmCnt + (size_t)kMaxG * 4;                      // int4 [kMaxG]: list offsets
-constexpr size_t kSmWsum = kSmLoff + (size_t)kMaxG * 16;                    // int4 [kMmaWarps]
+constexpr size_t kSmWsum = kSmLoff + (size_t)kMaxG * 16;                    // int4 [kWarps]
 static_assert(kSmBytes <= 227 * 1024, "shared memory");
+static_assert((size_t)kFixParts * kTile * 4 <= kSmS, "the split-K staging fits below the s/z rows");
 static_assert((size_t)kXCache * 2 <= (size_t)(kRing - kXSlot) * kStageBytes, "x cache fits");
-static_assert(kSmWsum + kMmaWarps * 16 <= kSmX, "output-CTA arrays below the x cache");
+static_assert(kSmWsum + kWarps * 16 <= kSmX, "output-CTA arrays below the x cache");
 static_assert(kSmRing % 16 == 0 && kSmX % 16 == 0 && kSmS % 16 == 0 && kSmZ % 16 == 0 &&
                   kSmBfrag % 16 == 0 && kSmLoff % 16 == 0 && kSmSlot % 16 == 0 &&
                   kSmWsum % 16 == 0 && kSmRed % 16 == 0 && kSmChunkCnt % 16 == 0 &&
-                  kSmWarpSum % 16 == 0 && kSmWarpBal % 16 == 0 && kSmWarpOff % 16 == 0 &&
-                  kSmBar % 8 == 0 && (kRow * 4) % 16 == 0,
-              "aligned regions (16 bytes for bulk copies and vector accesses, 8 for mbarriers)");
-static_assert((kStage * 16) % kCopyThreads == 0, "whole 16-byte copies per copy thread and stage");
-static_assert(kStage % (2 * kK) == 0 && kMmaWarps == 2 * kBlocks, "k-steps split between two warps");
-static_assert(kMaxG == kMmaThreads, "one group per thread in the output CTAs' scan");
-static_assert(kGroup == 4 * kChunkRows && kMmaWarps == 2 * kSlots, "two warps per slot, two chunks each");
-static_assert(kTile / 4 <= kThreads, "one float4 of a tile per thread in the split-K sums");
+                  kSmWarpSum % 16 == 0 && kSmWarpBal % 16 == 0 && kSmWarpOff % 16 == 0,
+              "16-byte aligned regions");
+static_assert((kStage * 16) % kThreads == 0, "whole 16-byte copies per thread and stage");
+static_assert(kStage % (2 * kK) == 0 && kWarps == 2 * kBlocks, "k-steps split between two warps");
+static_assert(kMaxG == kThreads, "one group per thread in the output CTAs' scan");
+static_assert(kGroup == 4 * kChunkRows && kWarps == 2 * kSlots, "two warps per slot, two chunks each");
 
 struct SlotInfo {
   int c;       // the group's B-column scale exponent: B holds x 4^(P-1-p) 2^-c
@@ -138,16 +130,15 @@ struct DecodeArgs {
   const float *theta;
   const float *phi;  // may be null: the default table
   int d_in, d_out, b_max, P, W, G, tiles;
-  int m;              // CTAs per tile (1: each CTA takes whole tiles in turn)
-  int cl;             // 1: the tile's CTAs add their partials inside their clusters first
   float *y;
   uint8_t *b;         // optional outputs (null: not written)
   int32_t *lists;
   int32_t *counts;
   float *grp_sums;
-  unsigned long long *counters;  // arrival words (count << 32 | arrival bits), left zero
+  unsigned *counters;  // arrival words (count | gave-up mark), left zero by every launch
   float *partials;    // [CTAs of this linear][kTile]
   int *error;         // the workspace's device error word
+  int m;              // CTAs per tile (1: each CTA takes whole tiles in turn)
   int reserve_out;    // set aside the output CTAs (the single call does, whether or not
                       // outputs are asked for, so y never depends on it; a group does not)
 };
@@ -162,8 +153,7 @@ struct DecodeGroup {
 // The optional outputs (b, lists, counts, group sums): written by CTAs that
 // take no part in the GEMV, so they cost the GEMV nothing but those CTAs' SMs.
 // Every output CTA counts the units of every group per plane and scans them
-// (the list offsets); then CTA k of K writes the groups g = k mod K.  Run by
-// the MMA warps of the CTA (kMmaThreads threads).
+// (the list offsets); then CTA k of K writes the groups g = k mod K.
 __device__ __forceinline__ void write_outputs(const DecodeArgs &a, unsigned char *smem, int k,
                                               int K, const __half2 (&t2)[4],
                                               const float (&phi)[5]) {
@@ -183,14 +173,14 @@ __device__ __forceinline__ void write_outputs(const DecodeArgs &a, unsigned char
   // units per (group, plane), x in chunks of kXCache rows
   for (int base = 0; base < a.d_in; base += kXCache) {
     const int rows = min(kXCache, a.d_in - base);
-    if (base > 0) sync_first<kMmaThreads>();
-    for (int q = tid; q < rows / 8; q += kMmaThreads) cp_async16(xc + 8 * q, a.x + base + 8 * q, 16);
+    if (base > 0) __syncthreads();
+    for (int q = tid; q < rows / 8; q += kThreads) cp_async16(xc + 8 * q, a.x + base + 8 * q, 16);
     cp_async_commit();
     cp_async_wait<0>();
-    sync_first<kMmaThreads>();
+    __syncthreads();
     xc_base = base;
     const int g_lo = base / kGroup, g_hi = (base + rows) / kGroup;
-    for (int g0 = g_lo; g0 < g_hi; g0 += kMmaThreads / kGT) {
+    for (int g0 = g_lo; g0 < g_hi; g0 += kThreads / kGT) {
       const int g = g0 + (tid >> 4);
       uint32_t mk[4] = {0u, 0u, 0u, 0u};
       if (g < g_hi) plane_masks8(load8(g), t2, P, mk);
@@ -202,10 +192,10 @@ __device__ __forceinline__ void write_outputs(const DecodeArgs &a, unsigned char
       if (gsub == 0 && g < g_hi) s_cnt[g] = packed;
     }
   }
-  sync_first<kMmaThreads>();
+  __syncthreads();
   // exclusive scans over groups: per-plane list offsets
   {
-    const int g0 = tid;  // kMaxG = kMmaThreads
+    const int g0 = tid;  // kMaxG = kThreads
     const uint32_t v = g0 < G ? s_cnt[g0] : 0u;
     const int4 v0 = make_int4(v & 255u, (v >> 8) & 255u, (v >> 16) & 255u, v >> 24);
     int4 inc = v0;
@@ -219,10 +209,10 @@ __device__ __forceinline__ void write_outputs(const DecodeArgs &a, unsigned char
       if (lane >= off) inc = make_int4(inc.x + t.x, inc.y + t.y, inc.z + t.z, inc.w + t.w);
     }
     if (lane == 31) s_wsum[warp] = inc;
-    sync_first<kMmaThreads>();
+    __syncthreads();
     int4 pre = make_int4(0, 0, 0, 0), tot = pre;
 #pragma unroll
-    for (int w = 0; w < kMmaWarps; ++w) {
+    for (int w = 0; w < kWarps; ++w) {
       const int4 t = s_wsum[w];
       if (w < warp) pre = make_int4(pre.x + t.x, pre.y + t.y, pre.z + t.z, pre.w + t.w);
       tot = make_int4(tot.x + t.x, tot.y + t.y, tot.z + t.z, tot.w + t.w);
@@ -236,10 +226,10 @@ __device__ __forceinline__ void write_outputs(const DecodeArgs &a, unsigned char
       if (P > 2) a.counts[2] = tot.z;
       if (P > 3) a.counts[3] = tot.w;
     }
-    sync_first<kMmaThreads>();
+    __syncthreads();
   }
   // team t (16 threads) of output CTA k writes group k + K (t + 32 pass)
-  for (int g0 = 0; g0 + k < G; g0 += K * (kMmaThreads / kGT)) {
+  for (int g0 = 0; g0 + k < G; g0 += K * (kThreads / kGT)) {
     const int g = g0 + k + K * (tid >> 4);
     const bool act = g < G;
     const uint4 xw = act ? load8(g) : make_uint4(0, 0, 0, 0);
@@ -297,16 +287,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
   uint16_t *z_st = reinterpret_cast<uint16_t *>(smem + kSmZ);
   SlotInfo *s_slot = reinterpret_cast<SlotInfo *>(smem + kSmSlot);
   float *s_red = reinterpret_cast<float *>(smem + kSmRed);
-  uint64_t *full = reinterpret_cast<uint64_t *>(smem + kSmBar);
-  uint64_t *empty = full + kRing;
-  uint64_t *sz_bar = empty + kRing;
   int *s_misc = reinterpret_cast<int *>(smem + kSmMisc);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const bool mma = warp < kMmaWarps;        // warp-uniform; the last kCopyWarps warps copy
   const int fg = lane >> 2, tq = lane & 3;  // MMA fragment row group and column pair
   const int ob = warp & (kBlocks - 1);      // the warp's 128-output block of the tile
-  const int kp = (warp / kBlocks) & 1;      // ... and its k-step parity
+  const int kp = warp / kBlocks;            // ... and its k-step parity
   // this CTA's linear, and the CTAs that linear has (a single linear: a fixed index,
   // so its arguments are read at fixed offsets)
   int jl = 0;
@@ -337,16 +323,20 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
   const int g_first = row_lo / kGroup;
   auto window_groups = [&](int g_w) { return min(kSlots, (row_hi + kGroup - 1) / kGroup - g_w); };
 
-  if (tid == 0) {
+  // the s and z rows of a window's groups for a tile, to shared memory (past d_out: zero)
+  auto stage_sz = [&](int tile, int g_w, int ng) {
 #pragma unroll
-    for (int i = 0; i < kRing; ++i) {
-      mbar_init(&full[i], kCopyThreads);  // one arrival per copy thread
-      mbar_init(&empty[i], kMmaWarps);    // one arrival per MMA warp
+    for (int i = 0; i < 2 * kSlots * (kTile / 8) / kThreads; ++i) {
+      const int q = tid + i * kThreads;  // [which][slot][chunk of 8 halves]
+      const int which = q / (kSlots * (kTile / 8)), gi = (q / (kTile / 8)) % kSlots;
+      const int ci = q % (kTile / 8), o = tile * kTile + ci * 8;
+      if (gi < ng) {
+        const uint16_t *src = (which ? a.z : a.s) + (size_t)(g_w + gi) * a.d_out + o;
+        uint16_t *dst = (which ? z_st : s_st) + gi * kTile + ci * 8;
+        cp_async16(dst, o < a.d_out ? (const void *)src : (const void *)a.s, o < a.d_out ? 16 : 0);
+      }
     }
-    mbar_init(sz_bar, 1);
-    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
-    asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
-  }
+  };
 
   // ---- theta and phi are not written by the kernel launched just before (a
   // condition of the call), so they are fetched before waiting for it; x, planes,
@@ -366,28 +356,20 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
   sort_thresholds(th_raw, t2);
 
   if (c >= C_g) {
-    if (mma && (a.b || a.lists || a.counts || a.grp_sums))
-      write_outputs(a, smem, c - C_g, n_out, t2, phi);
+    if (a.b || a.lists || a.counts || a.grp_sums) write_outputs(a, smem, c - C_g, n_out, t2, phi);
     return;
   }
-  if (c >= C_eff) return;  // (whole clusters: the host makes C_eff a multiple of the cluster size)
-  __syncthreads();         // the mbarriers are initialised
+  if (c >= C_eff) return;
+
+  for (int q = tid; q < kTile; q += kThreads) s_red[q] = 0.0f;  // (the first window's barrier orders it)
 
   int *s_ccnt = reinterpret_cast<int *>(smem + kSmChunkCnt);
   float4 *s_wsum = reinterpret_cast<float4 *>(smem + kSmWarpSum);
   uint4 *s_wbal = reinterpret_cast<uint4 *>(smem + kSmWarpBal);
   int4 *s_woff = reinterpret_cast<int4 *>(smem + kSmWarpOff);
 
-  uint64_t policy = 0;  // the copy warps' L2 policy: planes, s and z are read once
-  if (!mma) asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;\n" : "=l"(policy));
-
-  uint32_t gstage = 0;   // ring stages so far (every thread keeps the same count)
-  uint32_t sz_phase = 0; // s/z stagings so far
-  bool ok = true;
-
   for (int tile = tile_first; tile < a.tiles; tile += tile_step) {
-    const int wbase = tile * kTileW;                 // first word of the tile in a plane region
-    const int seg_words = min(kTileW, a.W - wbase);  // words of a unit's segment (ragged last tile)
+    const int wbase = tile * kTileW;  // first word of the tile in a plane region
     float yacc[16];
 #pragma unroll
     for (int t = 0; t < 16; ++t) yacc[t] = 0.0f;
@@ -398,79 +380,70 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
       if (g_w != g_first || tile != tile_first)
         __syncthreads();  // the previous window no longer reads the staged data
 
+      // ---- compaction, one row per lane: warp w takes chunks cc = 2 (w mod 2) and
+      // 2 (w mod 2) + 1 (32 rows each) of group slot w / 2, for every plane.  The
+      // window's units are ordered by slot, plane, chunk, row (any order works
+      // within a round: each unit carries its slot into B) ----
       const int slot = warp >> 1, cc0 = 2 * (warp & 1);
-      const bool live = mma && slot < ng;  // warp-uniform
+      const bool live = slot < ng;  // warp-uniform
       const int row0 = (g_w + slot) * kGroup + kChunkRows * cc0 + lane;  // the lane's row in chunk cc0
-      uint32_t xr = 0u;  // the lane's two x values (fp16 pair)
+      uint32_t xr = 0u, inb = 0u;  // the lane's two x values (fp16 pair) and which are in the slice
       uint32_t bal[2][4] = {{0u, 0u, 0u, 0u}, {0u, 0u, 0u, 0u}};
-      if (warp == kMmaWarps) {
-        // ---- copy warp 0: the s and z rows of the window's groups for this tile (the
-        // buffers of the previous window are free once its staging has landed) ----
-        if (sz_phase > 0) ok &= mbar_wait(sz_bar, (sz_phase - 1) & 1u, a.error);
-        if (lane == 0) mbar_arrive_expect_tx(sz_bar, (uint32_t)(2 * ng * seg_words * 32));
-        __syncwarp();
-        if (lane < 2 * ng) {
-          const int which = lane & 1, gi = lane >> 1;
-          const uint16_t *src = (which ? a.z : a.s) + (size_t)(g_w + gi) * a.d_out + tile * kTile;
-          bulk_g2s((which ? z_st : s_st) + gi * kTile, src, (uint32_t)seg_words * 32, sz_bar, policy);
+      if (live) {
+#pragma unroll
+        for (int ci = 0; ci < 2; ++ci) {
+          const int row = row0 + kChunkRows * ci;
+          if (row >= row_lo && row < row_hi) {
+            xr |= (uint32_t)__ldg(a.x + row) << (16 * ci);
+            inb |= 1u << ci;
+          }
         }
-      } else if (mma) {
-        // ---- compaction, one row per lane: warp w takes chunks cc = 2 (w mod 2) and
-        // 2 (w mod 2) + 1 (32 rows each) of group slot w / 2, for every plane.  The
-        // window's units are ordered by slot, plane, chunk, row (any order works
-        // within a round: each unit carries its slot into B) ----
-        uint32_t inb = 0u;  // which of the lane's two rows are in the slice
-        if (live) {
-#pragma unroll
-          for (int ci = 0; ci < 2; ++ci) {
-            const int row = row0 + kChunkRows * ci;
-            if (row >= row_lo && row < row_hi) {
-              xr |= (uint32_t)__ldg(a.x + row) << (16 * ci);
-              inb |= 1u << ci;
-            }
-          }
-          // plane p of a row is loaded when b > 2p, i.e. |x| >= the p-th smallest threshold
-          float X = 0.0f, Phi = 0.0f;
-          uint32_t amax = 0u;
-#pragma unroll
-          for (int ci = 0; ci < 2; ++ci) {
-            const uint32_t xb = (xr >> (16 * ci)) & 0xffffu;
-            const __half ax = __ushort_as_half((uint16_t)(xb & 0x7fffu));
-            int lev = 0;
-#pragma unroll
-            for (int p = 0; p < 4; ++p) {
-              const bool act = ((inb >> ci) & 1u) && __hge(ax, __low2half(t2[p]));
-              bal[ci][p] = __ballot_sync(0xffffffffu, act);
-              lev += act ? 1 : 0;
-            }
-            if (lev > 0) {
-              const float xv = __half2float(__ushort_as_half((uint16_t)xb));
-              X += xv;
-              Phi = __fmaf_rn(xv, pick_phi(phi, lev), Phi);
-              amax = max(amax, xb & 0x7fffu);
-            }
-          }
-#pragma unroll
-          for (int off = 16; off > 0; off >>= 1) {
-            X += __shfl_xor_sync(0xffffffffu, X, off);
-            Phi += __shfl_xor_sync(0xffffffffu, Phi, off);
-          }
-          amax = __reduce_max_sync(0xffffffffu, amax);
-          if (lane == 0) s_wsum[warp] = make_float4(X, Phi, __uint_as_float(amax), 0.0f);
-        }
-        // units per (slot, plane, chunk); lanes 0-7 write the warp's eight
-#pragma unroll
-        for (int ci = 0; ci < 2; ++ci)
-#pragma unroll
-          for (int p = 0; p < 4; ++p)
-            if (lane == 4 * ci + p) s_ccnt[(4 * slot + p) * 4 + cc0 + ci] = __popc(bal[ci][p]);
       }
+      // s and z are needed only at the flush: their copies go out after the x loads
+      stage_sz(tile, g_w, ng);
+      cp_async_commit();
+      if (live) {
+        // plane p of a row is loaded when b > 2p, i.e. |x| >= the p-th smallest threshold
+        float X = 0.0f, Phi = 0.0f;
+        uint32_t amax = 0u;
+#pragma unroll
+        for (int ci = 0; ci < 2; ++ci) {
+          const uint32_t xb = (xr >> (16 * ci)) & 0xffffu;
+          const __half ax = __ushort_as_half((uint16_t)(xb & 0x7fffu));
+          int lev = 0;
+#pragma unroll
+          for (int p = 0; p < 4; ++p) {
+            const bool act = ((inb >> ci) & 1u) && __hge(ax, __low2half(t2[p]));
+            bal[ci][p] = __ballot_sync(0xffffffffu, act);
+            lev += act ? 1 : 0;
+          }
+          if (lev > 0) {
+            const float xv = __half2float(__ushort_as_half((uint16_t)xb));
+            X += xv;
+            Phi = __fmaf_rn(xv, pick_phi(phi, lev), Phi);
+            amax = max(amax, xb & 0x7fffu);
+          }
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+          X += __shfl_xor_sync(0xffffffffu, X, off);
+          Phi += __shfl_xor_sync(0xffffffffu, Phi, off);
+        }
+        amax = __reduce_max_sync(0xffffffffu, amax);
+        if (lane == 0) s_wsum[warp] = make_float4(X, Phi, __uint_as_float(amax), 0.0f);
+      }
+      // units per (slot, plane, chunk); lanes 0-7 write the warp's eight
+#pragma unroll
+      for (int ci = 0; ci < 2; ++ci)
+#pragma unroll
+        for (int p = 0; p < 4; ++p)
+          if (lane == 4 * ci + p) s_ccnt[(4 * slot + p) * 4 + cc0 + ci] = __popc(bal[ci][p]);
       __syncthreads();
 
-      // exclusive prefix over the (slot, plane, chunk) counts (every MMA warp the
-      // same): lane L holds the four chunks of (slot, plane) = (L / 4, L mod 4)
-      int Nw = 0, cg = 0;
-      if (mma) {
+      // exclusive prefix over the (slot, plane, chunk) counts: lane L holds the four
+      // chunks of (slot, plane) = (L / 4, L mod 4)
+      int Nw;
+      {
         const int4 cv = reinterpret_cast<const int4 *>(s_ccnt)[lane];
         const int t = cv.x + cv.y + cv.z + cv.w;
         int inc = t;
@@ -495,30 +468,36 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
           s_woff[2 * warp] = make_int4(offv[0][0], offv[0][1], offv[0][2], offv[0][3]);
           s_woff[2 * warp + 1] = make_int4(offv[1][0], offv[1][1], offv[1][2], offv[1][3]);
         }
-        // the slot's B-column scale exponent: the largest active |x| of the slot, times
-        // 4^(P-1), stays below 2^16; and its group sums (for the flush)
-        if (live) {
-          const float4 w0 = s_wsum[2 * slot], w1 = s_wsum[2 * slot + 1];
-          const uint32_t am = max(__float_as_uint(w0.z), __float_as_uint(w1.z));
-          cg = (am >= 0x7c00u) ? 0 : max(0, (int)(am >> 10) - 15 + 2 * P - 16);
-          if (cc0 == 0 && lane == 0) {
-            SlotInfo si;
-            si.c = cg;
-            si.X = w0.x + w1.x;
-            si.Phi = w0.y + w1.y;
-            si.pad = 0;
-            s_slot[slot] = si;
-          }
-        }
-        if (warp == 0 && lane == 0) s_misc[0] = Nw;
-        __syncwarp();
       }
+      // the slot's B-column scale exponent: the largest active |x| of the slot, times
+      // 4^(P-1), stays below 2^16; and its group sums (for the flush)
+      int cg = 0;
+      if (live) {
+        const float4 w0 = s_wsum[2 * slot], w1 = s_wsum[2 * slot + 1];
+        const uint32_t am = max(__float_as_uint(w0.z), __float_as_uint(w1.z));
+        cg = (am >= 0x7c00u) ? 0 : max(0, (int)(am >> 10) - 15 + 2 * P - 16);
+        if (cc0 == 0 && lane == 0) {
+          SlotInfo si;
+          si.c = cg;
+          si.X = w0.x + w1.x;
+          si.Phi = w0.y + w1.y;
+          si.pad = 0;
+          s_slot[slot] = si;
+        }
+      }
+      __syncwarp();
 
-      // the records of the MMA warp's units that fall in [k0, k0 + n): plane region and
-      // x 4^(P-1-p) 2^-c rounded to fp16 (a power-of-two product: exact unless the
-      // result is subnormal, then rounded as fp16 does) with the slot; padding units
-      // (to whole stages) load nothing and have B = 0
-      auto write_records = [&](int k0, int n, int n_pad) {
+      for (int k0 = 0; k0 < Nw; k0 += kRound) {
+        // the round is padded to whole stages with units whose B entries are 0 and
+        // which load nothing: every warp runs every k-step of a stage unconditionally
+        const int n = min(kRound, Nw - k0), n_pad = (n + kStage - 1) & ~(kStage - 1);
+        const int n_steps = n_pad / kK, n_stages = n_pad / kStage;
+        static_assert(kRound % kStage == 0, "rounds of whole stages");
+        if (k0 > 0) __syncthreads();  // the previous round no longer reads the records
+
+        // the records of the warp's units that fall in [k0, k0 + n): plane region
+        // and x 4^(P-1-p) 2^-c rounded to fp16 (a power-of-two product: exact unless
+        // the result is subnormal, then rounded as fp16 does) with the slot
         if (live) {
           const uint32_t lt = (1u << lane) - 1u;
 #pragma unroll
@@ -540,70 +519,18 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
             }
           }
         }
-        for (int k = n + tid; k < n_pad; k += kMmaThreads) {
+        for (int k = n + tid; k < n_pad; k += kThreads) {  // padding units: no load, B = 0
           s_region[k] = -1;
           s_ux[k] = 0u;
         }
-      };
-      auto round_size = [](int Nw_, int k0, int &n, int &n_pad) {
-        n = min(kRound, Nw_ - k0);
-        n_pad = (n + kStage - 1) & ~(kStage - 1);
-      };
-      if (mma && Nw > 0) {
-        int n, n_pad;
-        round_size(Nw, 0, n, n_pad);
-        write_records(0, n, n_pad);
-      }
-      __syncthreads();
-      Nw = s_misc[0];
+        __syncthreads();
 
-      for (int k0 = 0; k0 < Nw; k0 += kRound) {
-        // the round is padded to whole stages with units whose B entries are 0 and
-        // which load nothing: every warp runs every k-step of a stage unconditionally
-        int n, n_pad;
-        round_size(Nw, k0, n, n_pad);
-        const int n_steps = n_pad / kK, n_stages = n_pad / kStage;
-        static_assert(kRound % kStage == 0, "rounds of whole stages");
-        if (k0 > 0) {
-          __syncthreads();  // the previous round no longer reads the records
-          if (mma) write_records(k0, n, n_pad);
-          __syncthreads();
-        }
-
-        if (!mma) {
-          // ---- copy warps: copy thread ct takes the 16-byte pieces ct + kCopyThreads j of
-          // the stage (a warp's 32 lanes: two units' 256-byte segments) ----
-          const int ct = tid - kMmaThreads;
-          for (int st = 0; st < n_stages; ++st) {
-            const uint32_t gs = gstage + st, rs = gs % kRing;
-            if (gs >= kRing) ok &= mbar_wait(&empty[rs], ((gs / kRing) - 1u) & 1u, a.error);
-            uint32_t *dst_stage = ring + (size_t)rs * (kStage * kRow);
-#pragma unroll
-            for (int j = 0; j < kStage * 16 / kCopyThreads; ++j) {
-              const int q = ct + kCopyThreads * j, ul = q >> 4, part16 = q & 15;
-              const int region = s_region[st * kStage + ul];
-              const int word = 4 * part16;
-              if (region >= 0 && word < seg_words) {
-                const uint32_t *src = a.planes + (size_t)region * a.W + wbase + word;
-                uint32_t *dst = dst_stage + ul * kRow + word;
-                if (ALIGNED) {
-                  cp_async16_hint(dst, src, policy);
-                } else {
-#pragma unroll
-                  for (int v = 0; v < 4; ++v)
-                    if (word + v < seg_words) cp_async4(dst + v, src + v);
-                }
-              }
-            }
-            cp_async_mbar_arrive(&full[rs]);  // counts once this thread's copies have landed
-          }
-        } else {
-          // ---- MMA warps ----
-          // B fragments per k-step: lane (fg, tq) holds B[2tq, 2tq+1][fg] and B[2tq+8, 2tq+9][fg];
-          // B[k][col] = x'' of unit k if the unit's group slot is col / 2 + 4 (col mod 2), else
-          // 0.  So D column 2q holds slot q and column 2q+1 slot q+4, and a window of at
-          // most 4 groups leaves the second slot of every lane empty (skipped by the flush)
-          for (int q = tid; q < n_steps * 32; q += kMmaThreads) {
+        // B fragments per k-step: lane (fg, tq) holds B[2tq, 2tq+1][fg] and B[2tq+8, 2tq+9][fg];
+        // B[k][col] = x'' of unit k if the unit's group slot is col / 2 + 4 (col mod 2), else
+        // 0.  So D column 2q holds slot q and column 2q+1 slot q+4, and a window of at
+        // most 4 groups leaves the second slot of every lane empty (skipped by the flush)
+        auto build_bfrag = [&]() {
+          for (int q = tid; q < n_steps * 32; q += kThreads) {
             const int kk = q >> 5, L = q & 31, col = L >> 2, t2i = 2 * (L & 3);
             const int slot_c = (col >> 1) + 4 * (col & 1);
             const uint32_t *ux = s_ux + kk * kK;
@@ -611,34 +538,31 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
             s_bfrag[q] = make_uint2(bh(ux[t2i]) | (bh(ux[t2i + 1]) << 16),
                                     bh(ux[t2i + 8]) | (bh(ux[t2i + 9]) << 16));
           }
-          sync_first<kMmaThreads>();
+        };
 
-          float d[8][4];
+        float d[8][4];
 #pragma unroll
-          for (int bk = 0; bk < 8; ++bk) d[bk][0] = d[bk][1] = d[bk][2] = d[bk][3] = 0.0f;
+        for (int bk = 0; bk < 8; ++bk) d[bk][0] = d[bk][1] = d[bk][2] = d[bk][3] = 0.0f;
 
-          for (int st = 0; st < n_stages; ++st) {
-            const uint32_t gs = gstage + st, rs = gs % kRing;
-            ok &= mbar_wait(&full[rs], (gs / kRing) & 1u, a.error);
-            // this warp's k-steps h = kp and kp + 2 of the stage, operands of both first
-            constexpr int kStepsPerWarp = kStage / kK / 2;
-            const uint32_t *sb = ring + (size_t)rs * (kStage * kRow);
-            uint32_t wv[kStepsPerWarp][4];
-            uint2 bv[kStepsPerWarp];
+        // this warp's MMA work on ring stage st (units 64 st .. 64 st + 63 of the round,
+        // held in `sb`): its k-steps h = kp and kp + 2, operands of both first
+        constexpr int kStepsPerWarp = kStage / kK / 2;  // k-steps of a stage per warp
+        auto compute = [&](const uint32_t *sb, int st) {
+          uint32_t wv[kStepsPerWarp][4];
+          uint2 bv[kStepsPerWarp];
 #pragma unroll
-            for (int i = 0; i < kStepsPerWarp; ++i) {
-              const int h = kp + 2 * i, kk = kStage / kK * st + h;
-              const uint32_t *pw = sb + (h * kK + 2 * tq) * kRow + 8 * ob + fg;
-              wv[i][0] = pw[0];
-              wv[i][1] = pw[kRow];
-              wv[i][2] = pw[8 * kRow];
-              wv[i][3] = pw[9 * kRow];
-              bv[i] = s_bfrag[kk * 32 + lane];
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[rs]);  // the stage's words are in registers
+          for (int i = 0; i < kStepsPerWarp; ++i) {
+            const int h = kp + 2 * i, kk = kStage / kK * st + h;
+            const uint32_t *pw = sb + (h * kK + 2 * tq) * kRow + 8 * ob + fg;
+            wv[i][0] = pw[0];
+            wv[i][1] = pw[kRow];
+            wv[i][2] = pw[8 * kRow];
+            wv[i][3] = pw[9 * kRow];
+            bv[i] = s_bfrag[kk * 32 + lane];
+          }
 #pragma unroll
-            for (int i = 0; i < kStepsPerWarp; ++i) {
+          for (int i = 0; i < kStepsPerWarp; ++i) {
+            {
               const uint32_t w0 = wv[i][0], w1 = wv[i][1], w2 = wv[i][2], w3 = wv[i][3];
               const uint2 bb = bv[i];
               // m0/m1: outputs 0-7 / 8-15 of units 2tq (low half) and 2tq+1 (high half);
@@ -658,89 +582,117 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
               mma16816(d[7], n1 & (F << 6), n1 & (F << 8), n3 & (F << 6), n3 & (F << 8), bb.x, bb.y);
             }
           }
+        };
 
-          // flush: y_t += s (D 2^(24 - pos(t) + c) [+ Phi]) [+ z X] for the lane's two slots
-          // (tq and tq + 4); the slice's group terms once per window (first round, even-k warps)
-          ok &= mbar_wait(sz_bar, sz_phase & 1u, a.error);
-          const bool terms = k0 == 0 && kp == 0;
+        // ---- cp.async ring: 16 threads copy a unit's segment (16-byte copies; 4-byte
+        // copies for layouts whose rows are not 16-byte aligned) ----
+        auto issue = [&](int st) {
+          uint32_t *dst_stage = ring + (size_t)(st % kRing) * (kStage * kRow);
 #pragma unroll
-          for (int jj = 0; jj < 2; ++jj) {
-            const int j = tq + 4 * jj;
-            if (j < ng) {
-              const SlotInfo si = s_slot[j];
-              const uint16_t *srow = s_st + j * kTile + 128 * ob + 16 * fg;
-              const uint16_t *zrow = z_st + j * kTile + 128 * ob + 16 * fg;
-              float sv[16], zv[16];
-              const uint4 s0 = *reinterpret_cast<const uint4 *>(srow);
-              const uint4 s1 = *reinterpret_cast<const uint4 *>(srow + 8);
-              const uint4 z0 = *reinterpret_cast<const uint4 *>(zrow);
-              const uint4 z1 = *reinterpret_cast<const uint4 *>(zrow + 8);
-              const uint32_t su[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
-              const uint32_t zu[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
+          for (int h = 0; h < kStage * 16 / kThreads; ++h) {
+            const int q = tid + h * kThreads, ul = q >> 4, part16 = q & 15;
+            const int k = st * kStage + ul;
+            const int region = k < n_pad ? s_region[k] : -1;
+            const int word = wbase + part16 * 4;
+            uint32_t *dst = dst_stage + ul * kRow + part16 * 4;
+            if (region >= 0) {
+              const uint32_t *src = a.planes + (size_t)region * a.W + word;
+              if (ALIGNED) {
+                if (word < a.W) cp_async16(dst, src, 16);
+              } else {
 #pragma unroll
-              for (int k = 0; k < 8; ++k) {
-                const float2 fs = __half22float2(*reinterpret_cast<const __half2 *>(&su[k]));
-                const float2 fz = __half22float2(*reinterpret_cast<const __half2 *>(&zu[k]));
-                sv[2 * k] = fs.x;
-                sv[2 * k + 1] = fs.y;
-                zv[2 * k] = fz.x;
-                zv[2 * k + 1] = fz.y;
-              }
-#pragma unroll
-              for (int bk = 0; bk < 8; ++bk) {
-                const int t0 = 2 * bk, t1 = 2 * bk + 1;
-                float v0 = d[bk][jj] * exp2i(24 - field_pos(t0) + si.c);
-                float v1 = d[bk][2 + jj] * exp2i(24 - field_pos(t1) + si.c);
-                if (terms) {
-                  v0 += si.Phi;
-                  v1 += si.Phi;
-                  yacc[t0] = fmaf(zv[t0], si.X, yacc[t0]);
-                  yacc[t1] = fmaf(zv[t1], si.X, yacc[t1]);
-                }
-                yacc[t0] = fmaf(sv[t0], v0, yacc[t0]);
-                yacc[t1] = fmaf(sv[t1], v1, yacc[t1]);
+                for (int v = 0; v < 4; ++v)
+                  if (word + v < a.W) cp_async4(dst + v, src + v);
               }
             }
           }
+        };
+#pragma unroll
+        for (int st = 0; st < kRing - 1; ++st) {
+          if (st < n_stages) issue(st);
+          cp_async_commit();
         }
-        gstage += (uint32_t)n_stages;
+        build_bfrag();
+        for (int st = 0; st < n_stages; ++st) {
+          cp_async_wait<kRing - 2>();  // this thread's copies of stage st (and s/z) landed
+          __syncthreads();             // everybody's; and stage st-1 is no longer read
+          if (st + kRing - 1 < n_stages) issue(st + kRing - 1);
+          cp_async_commit();
+          compute(ring + (size_t)(st % kRing) * (kStage * kRow), st);
+        }
+        cp_async_wait<0>();
+
+        // flush: y_t += s (D 2^(24 - pos(t) + c) [+ Phi]) [+ z X] for the lane's two slots
+        // (tq and tq + 4); the slice's group terms once per window (first round, even-k warps)
+        const bool terms = k0 == 0 && kp == 0;
+#pragma unroll
+        for (int jj = 0; jj < 2; ++jj) {
+          const int j = tq + 4 * jj;
+          if (j < ng) {
+            const SlotInfo si = s_slot[j];
+            const uint16_t *srow = s_st + j * kTile + 128 * ob + 16 * fg;
+            const uint16_t *zrow = z_st + j * kTile + 128 * ob + 16 * fg;
+            float sv[16], zv[16];
+            const uint4 s0 = *reinterpret_cast<const uint4 *>(srow);
+            const uint4 s1 = *reinterpret_cast<const uint4 *>(srow + 8);
+            const uint4 z0 = *reinterpret_cast<const uint4 *>(zrow);
+            const uint4 z1 = *reinterpret_cast<const uint4 *>(zrow + 8);
+            const uint32_t su[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+            const uint32_t zu[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+              const float2 fs = __half22float2(*reinterpret_cast<const __half2 *>(&su[k]));
+              const float2 fz = __half22float2(*reinterpret_cast<const __half2 *>(&zu[k]));
+              sv[2 * k] = fs.x;
+              sv[2 * k + 1] = fs.y;
+              zv[2 * k] = fz.x;
+              zv[2 * k + 1] = fz.y;
+            }
+#pragma unroll
+            for (int bk = 0; bk < 8; ++bk) {
+              const int t0 = 2 * bk, t1 = 2 * bk + 1;
+              float v0 = d[bk][jj] * exp2i(24 - field_pos(t0) + si.c);
+              float v1 = d[bk][2 + jj] * exp2i(24 - field_pos(t1) + si.c);
+              if (terms) {
+                v0 += si.Phi;
+                v1 += si.Phi;
+                yacc[t0] = fmaf(zv[t0], si.X, yacc[t0]);
+                yacc[t1] = fmaf(zv[t1], si.X, yacc[t1]);
+              }
+              yacc[t0] = fmaf(sv[t0], v0, yacc[t0]);
+              yacc[t1] = fmaf(sv[t1], v1, yacc[t1]);
+            }
+          }
+        }
       }
-      ++sz_phase;
     }
 
-    // ---- the CTA's partial tile: the 4 lanes of a quad (their slots), then the two
-    // k-parity warps of a block, into s_red ----
-    float fin[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-    if (mma) {
-      float keep[8];
+    // ---- reduce the 4 lanes of a quad (their slots); lane keeps 4 outputs ------
+    float keep[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const float send = (tq & 1) ? yacc[i] : yacc[8 + i];
-        const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
-        keep[i] = ((tq & 1) ? yacc[8 + i] : yacc[i]) + recv;
-      }
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float send = (tq & 2) ? keep[i] : keep[4 + i];
-        const float recv = __shfl_xor_sync(0xffffffffu, send, 2);
-        fin[i] = ((tq & 2) ? keep[4 + i] : keep[i]) + recv;
-      }
+    for (int i = 0; i < 8; ++i) {
+      const float send = (tq & 1) ? yacc[i] : yacc[8 + i];
+      const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
+      keep[i] = ((tq & 1) ? yacc[8 + i] : yacc[i]) + recv;
     }
-    const int ol = 128 * ob + 16 * fg + 8 * (tq & 1) + 4 * (tq >> 1);  // first of the lane's 4 outputs
+    float fin[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float send = (tq & 2) ? keep[i] : keep[4 + i];
+      const float recv = __shfl_xor_sync(0xffffffffu, send, 2);
+      fin[i] = ((tq & 2) ? keep[4 + i] : keep[i]) + recv;
+    }
+    const int ol = 128 * ob + 16 * fg + 8 * (tq & 1) + 4 * (tq >> 1);  // first of 4 outputs
     const int obase = tile * kTile;
-    __syncthreads();  // s_red of the previous tile is consumed
-    if (mma && kp == 1) *reinterpret_cast<float4 *>(s_red + ol) = make_float4(fin[0], fin[1], fin[2], fin[3]);
+    // the two k-parity warps of a block add into s_red (zero here): a sum of two values
+    // does not depend on their order, so the CTA's partial is deterministic
+#pragma unroll
+    for (int i = 0; i < 4; ++i) atomicAdd(s_red + ol + i, fin[i]);
     __syncthreads();
-    if (mma && kp == 0) {
-      const float4 o = *reinterpret_cast<const float4 *>(s_red + ol);
-      *reinterpret_cast<float4 *>(s_red + ol) =
-          make_float4(fin[0] + o.x, fin[1] + o.y, fin[2] + o.z, fin[3] + o.w);
-    }
-    __syncthreads();
-
     if (m == 1) {  // the whole tile's rows: y directly
       for (int q = tid; q < kTile / 4; q += kThreads) {
         const float4 v = reinterpret_cast<const float4 *>(s_red)[q];
+        reinterpret_cast<float4 *>(s_red)[q] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);  // for the next tile
         const int o = obase + 4 * q;  // d_out % 16 == 0: a float4 is wholly in or out
         if (o < a.d_out) {
           a.y[o] = v.x;
@@ -751,94 +703,84 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
       }
       continue;
     }
-
-    // ---- split-K.  The share this CTA sums or publishes: outputs [sh0, sh0 + nsh) of
-    // the tile.  With clusters: the cluster's CL partials first, CTA r of the
-    // cluster taking share r; then the m / CL cluster sums of share r meet in
-    // global memory.  Without: the m partials of the whole tile. ----
-    int cl_n = 1, rank = 0;
-    if (a.cl) {
-      asm("mov.u32 %0, %%cluster_nctarank;" : "=r"(cl_n));
-      rank = (int)cluster_rank();
-    }
-    const int nsh = kTile / cl_n, sh0 = rank * nsh;
-    float4 val = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-    const bool mine = tid < nsh / 4;  // the threads that hold a float4 of the share
-    if (a.cl) {
-      cluster_arrive();
-      cluster_wait();  // every CTA of the cluster has its partial in s_red
-      if (mine)
-        for (int k = 0; k < cl_n; ++k) val = f4add(val, ld_peer_f4(s_red + sh0 + 4 * tid, (uint32_t)k));
-      cluster_arrive();  // done reading the peers' s_red (waited for before exit)
-    } else if (mine) {
-      val = reinterpret_cast<const float4 *>(s_red)[tid];
-    }
-    const int npart = m / cl_n;  // sums that meet in global memory (1: none)
-    if (npart == 1) {
-      if (mine) {
-        const int o = obase + sh0 + 4 * tid;
-        if (o < a.d_out) {
-          a.y[o] = val.x;
-          a.y[o + 1] = val.y;
-          a.y[o + 2] = val.z;
-          a.y[o + 3] = val.w;
-        }
-      }
-    } else {
-      // publish, then count the arrival on the share's 64-bit arrival word: the
-      // count in the high half, and (up to 32 partials) a bit per publisher in the
-      // low half, both set by one atomic add.  The arrival that brings the count to
-      // npart sums the npart published values in a fixed order.  CTA (cluster k,
-      // rank r) of the tile is c_first + k cl_n + r.
-      const int c_first = (c / m) * m, kidx = (c - c_first) / cl_n;
-      if (mine) reinterpret_cast<float4 *>(a.partials + (size_t)c * kTile + sh0)[tid] = val;
-      __syncthreads();
-      if (tid == 0) {
-        unsigned long long *word = a.counters + (a.cl ? tile * cl_n + rank : tile);
-        const bool masked = npart <= 32;
-        const unsigned full = !masked ? 0u : npart == 32 ? 0xffffffffu : (1u << npart) - 1u;
-        const unsigned long long add = (1ull << 32) | (masked ? 1ull << kidx : 0ull);
-        __threadfence();  // the partial (ordered before by the barrier), then the count
-        const unsigned long long old = atomicAdd(word, add);
-        const bool last = (unsigned)(old >> 32) == (unsigned)(npart - 1);
-        if (last) {
-          // a count that did not start at zero (a workspace not left zeroed) makes
-          // this arrival come early: the arrival bits show who is missing; wait
-          // for them, report error 3, and leave the word clean
-          if (masked && (((unsigned)old | (unsigned)add) & full) != full) {
-            int polls = 0;
-            while ((unsigned)(ld_acquire64(word) & full) != full && ++polls < kFlagPolls)
-              __nanosleep(64);
-            atomicCAS(a.error, 0, kDevErrSplitKTimeout);
+    // ---- split-K: the m partial tiles of a tile meet in global memory.  Every CTA
+    // publishes its partial and counts its arrival on the tile's arrival word; once
+    // all m have arrived, every CTA adds up its own 1/m share of the outputs over the
+    // m partials in CTA order (deterministic), so the sum is spread over the tile's
+    // CTAs.  Waiting for the others needs them to be running; if one is not (the GPU
+    // is shared with other work), a waiter gives up after a bound, marks the word,
+    // and exits -- and the tile's last arrival, which sees that mark in the value its
+    // own arrival returns, then sums the whole tile itself.  So every output is
+    // written, by its owner or by the last arrival (the same bits either way). ----
+    const int c_first = (c / m) * m;
+    if (tid < kTile / 4)
+      reinterpret_cast<float4 *>(a.partials + (size_t)c * kTile)[tid] =
+          reinterpret_cast<const float4 *>(s_red)[tid];
+    __syncthreads();
+    if (tid == 0) {
+      unsigned *word = a.counters + tile;
+      asm volatile("fence.sc.gpu;\n" ::: "memory");  // the partial (ordered before by the barrier)
+      const unsigned old = atomicAdd(word, 1u);
+      const unsigned cnt = old & kCountMask;
+      int role;  // 0: sum the own share, 1: sum the whole tile, 2: gave up
+      if (cnt == (unsigned)(m - 1)) {  // the last arrival: bring the count back to zero
+        role = (old & kGaveUp) ? 1 : 0;
+        atomicSub(word, (unsigned)m);
+        if (role == 1) atomicAnd(word, ~kGaveUp);
+      } else {
+        // complete once the count reads m (the last arrival) or 0 (reset after it)
+        role = 2;
+        for (int polls = 0; polls < kSpinLimit; ++polls) {
+          const unsigned c2 = ld_acquire(word) & kCountMask;
+          if (c2 == 0u || c2 == (unsigned)m) {
+            role = 0;
+            break;
           }
-          __threadfence();  // the others' partials are visible to this CTA
-          *reinterpret_cast<volatile unsigned long long *>(word) = 0ull;
+          __nanosleep(32);
         }
-        s_misc[1] = last ? 1 : 0;
+        if (role == 2) {
+          // mark the word, then look once more: either the last arrival has come (and the
+          // mark is stale but harmless), or it has not and will see the mark
+          asm volatile("fence.sc.gpu;\n" ::: "memory");
+          const unsigned c2 = atomicOr(word, kGaveUp) & kCountMask;
+          if (c2 == 0u || c2 == (unsigned)m) role = 0;
+          else atomicCAS(a.error, 0, kDevErrSplitKTimeout);
+        }
       }
-      __syncthreads();
-      if (s_misc[1] && mine) {
-        float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-        for (int k = 0; k < npart; ++k)
-          acc = f4add(acc, __ldcg(reinterpret_cast<const float4 *>(
-                                      a.partials + (size_t)(c_first + k * cl_n + rank) * kTile + sh0) +
-                                  tid));
-        const int o = obase + sh0 + 4 * tid;
-        if (o < a.d_out) {
-          a.y[o] = acc.x;
-          a.y[o + 1] = acc.y;
-          a.y[o + 2] = acc.z;
-          a.y[o + 3] = acc.w;
+      asm volatile("fence.sc.gpu;\n" ::: "memory");  // the others' partials are visible
+      s_misc[1] = role;
+    }
+    __syncthreads();
+    const int role = s_misc[1];
+    if (role != 2) {
+      // the quads [Q k / m, Q (k + 1) / m) of share k, Q = kTile / 4: share `part`, or all
+      const int q0 = role == 1 ? 0 : (kTile / 4) * part / m;
+      const int nq = role == 1 ? kTile / 4 : (kTile / 4) * (part + 1) / m - q0;
+      float4 *stage = reinterpret_cast<float4 *>(smem);  // [parts][nq]: the idle ring
+      const int per_pass = nq == kTile / 4 ? kFixParts : m;
+      float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+      for (int k0 = 0; k0 < m; k0 += per_pass) {
+        const int np = min(per_pass, m - k0);
+        for (int q = tid; q < np * nq; q += kThreads) {
+          const int k = q / nq, qq = q - k * nq;
+          cp_async16(stage + q, a.partials + (size_t)(c_first + k0 + k) * kTile + 4 * (q0 + qq), 16);
         }
+        cp_async_commit();
+        cp_async_wait<0>();
+        __syncthreads();
+        if (tid < nq)
+          for (int k = 0; k < np; ++k) acc = f4add(acc, stage[k * nq + tid]);  // in CTA order
+        __syncthreads();
+      }
+      const int o = obase + 4 * (q0 + tid);
+      if (tid < nq && o < a.d_out) {
+        a.y[o] = acc.x;
+        a.y[o + 1] = acc.y;
+        a.y[o + 2] = acc.z;
+        a.y[o + 3] = acc.w;
       }
     }
-    if (a.cl) cluster_wait();  // the peers no longer read this CTA's s_red
   }
-
-  // copy warp 0 leaves no bulk copy in flight: the last s/z staging has landed (the
-  // ring's stages were all consumed by the MMA warps)
-  if (warp == kMmaWarps && sz_phase > 0) ok &= mbar_wait(sz_bar, (sz_phase - 1) & 1u, a.error);
-  (void)ok;
 }
 
 int device_sms() {
@@ -853,41 +795,8 @@ int device_sms() {
   return n;
 }
 
-// CTAs of a launch with clusters of `cl` that the device holds at once (at one
-// CTA per SM), queried once per device and cluster size.
 template <bool ALIGNED, bool GROUPED>
-int cluster_capacity(int cl) {
-  static int cached[64][5] = {{0}};
-  const int idx = cl == 2 ? 1 : cl == 4 ? 2 : 0;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return 0;
-  if (cached[dev][idx]) return cached[dev][idx] - 1;
-  int n = 0;
-  const void *fn = (const void *)decode_kernel<ALIGNED, GROUPED>;
-  if (ensure_smem_attr(fn, kSmBytes) == cudaSuccess) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(cl * 4);
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = kSmBytes;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = cl;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    int clusters = 0;
-    if (cudaOccupancyMaxActiveClusters(&clusters, decode_kernel<ALIGNED, GROUPED>, &cfg) == cudaSuccess)
-      n = clusters * cl;
-    else
-      (void)cudaGetLastError();
-  }
-  cached[dev][idx] = n + 1;
-  return n;
-}
-
-template <bool ALIGNED, bool GROUPED>
-cudaError_t launch_variant(const DecodeGroup &g, int cl, cudaStream_t st) {
+cudaError_t launch_variant(const DecodeGroup &g, cudaStream_t st) {
   cudaError_t e = ensure_smem_attr((const void *)decode_kernel<ALIGNED, GROUPED>, kSmBytes);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -895,21 +804,17 @@ cudaError_t launch_variant(const DecodeGroup &g, int cl, cudaStream_t st) {
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = kSmBytes;
   cfg.stream = st;
-  cudaLaunchAttribute attr[2];
+  cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
-  attr[1].id = cudaLaunchAttributeClusterDimension;
-  attr[1].val.clusterDim.x = cl;
-  attr[1].val.clusterDim.y = 1;
-  attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = cl > 1 ? 2 : 1;
+  cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, decode_kernel<ALIGNED, GROUPED>, g);
 }
 
 DecodeArgs make_args(const uint32_t *planes, const uint16_t *s, const uint16_t *z,
                      const uint16_t *x, const float *theta, const float *phi, int d_in, int d_out,
-                     int b_max, float *y) {
+                     int b_max, float *y, int n_gemv) {
   DecodeArgs a = {};
   a.planes = planes;
   a.s = s;
@@ -924,35 +829,16 @@ DecodeArgs make_args(const uint32_t *planes, const uint16_t *s, const uint16_t *
   a.W = d_out / 16;
   a.G = d_in / kGroup;
   a.tiles = (d_out + kTile - 1) / kTile;
+  a.m = a.tiles >= n_gemv ? 1 : n_gemv / a.tiles;  // CTAs per tile (1: whole tiles in turn)
   a.y = y;
   return a;
 }
 
-// Bytes the summing CTA of a split tile reads, for m CTAs per tile in clusters of cl
-// (the cost a cluster size is chosen by); 0 when every CTA has whole tiles.
-size_t split_read_bytes(int m, int cl) {
-  if (m <= 1) return 0;
-  const int npart = (cl > 1 && m % cl == 0) ? m / cl : m;
-  return npart > 1 ? (size_t)npart * (kTile / (m % cl == 0 ? cl : 1)) * 4 : 0;
-}
-
-// CTAs per tile and whether a linear's tiles add their partials in clusters of cl.
-void set_split(DecodeArgs &a, int n_gemv, int cl) {
-  if (a.tiles >= n_gemv) {
-    a.m = 1;
-    a.cl = 0;
-    return;
-  }
-  a.m = n_gemv / a.tiles;
-  a.cl = (cl > 1 && a.m % cl == 0) ? 1 : 0;
-}
-
 template <bool GROUPED>
-cudaError_t launch_group(DecodeGroup &g, int cl, cudaStream_t st) {
+cudaError_t launch_group(DecodeGroup &g, cudaStream_t st) {
   bool aligned = true;  // 16-byte plane copies need every linear's rows 16-byte aligned
   for (int j = 0; j < g.n; ++j) aligned = aligned && g.lin[j].W % 4 == 0;
-  cudaError_t e = aligned ? launch_variant<true, GROUPED>(g, cl, st)
-                          : launch_variant<false, GROUPED>(g, cl, st);
+  cudaError_t e = aligned ? launch_variant<true, GROUPED>(g, st) : launch_variant<false, GROUPED>(g, st);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
@@ -966,7 +852,7 @@ cudaError_t launch_decode(const uint32_t *planes, const uint16_t *s, const uint1
   const WsLayout L = ws_layout(d_in, d_out, b_max);
   char *w = static_cast<char *>(ws);
   return launch_decode_split(planes, s, z, x, theta, phi, d_in, d_out, b_max, y, b, lists, counts,
-                             grp_sums, reinterpret_cast<unsigned long long *>(w + L.counters),
+                             grp_sums, reinterpret_cast<unsigned *>(w + L.counters),
                              reinterpret_cast<float *>(w + L.partials),
                              &reinterpret_cast<WsHeader *>(w)->error, st);
 }
@@ -974,13 +860,16 @@ cudaError_t launch_decode(const uint32_t *planes, const uint16_t *s, const uint1
 cudaError_t launch_decode_split(const uint32_t *planes, const uint16_t *s, const uint16_t *z,
                                 const uint16_t *x, const float *theta, const float *phi, int d_in,
                                 int d_out, int b_max, float *y, uint8_t *b, int32_t *lists,
-                                int32_t *counts, float *grp_sums, unsigned long long *counters,
+                                int32_t *counts, float *grp_sums, unsigned *counters,
                                 float *partials, int *error, cudaStream_t st) {
   DecodeGroup g = {};
   g.n = 1;
   g.cta_start[0] = 0;
+  const int C = device_sms();
+  g.cta_start[1] = C;
   DecodeArgs &a = g.lin[0];
-  a = make_args(planes, s, z, x, theta, phi, d_in, d_out, b_max, y);
+  a = make_args(planes, s, z, x, theta, phi, d_in, d_out, b_max, y,
+                C - (C > 2 * kOutCtas ? kOutCtas : 1));
   a.b = b;
   a.lists = lists;
   a.counts = counts;
@@ -989,97 +878,49 @@ cudaError_t launch_decode_split(const uint32_t *planes, const uint16_t *s, const
   a.partials = partials;
   a.error = error;
   a.reserve_out = 1;
-  // the cluster size whose split reads the fewest bytes, among those whose clusters
-  // the device holds at once
-  const bool aligned = a.W % 4 == 0;
-  const int C = device_sms();
-  int best_cl = 1;
-  size_t best = ~size_t(0);
-  for (int cl : {4, 2, 1}) {
-    if (C % cl != 0) continue;
-    if (cl > 1 && (aligned ? cluster_capacity<true, false>(cl) : cluster_capacity<false, false>(cl)) < C)
-      continue;
-    const int n_out = C > 2 * kOutCtas ? kOutCtas : 1;
-    const int n_gemv = C - n_out;
-    if (n_out % cl != 0) continue;
-    DecodeArgs t = a;
-    set_split(t, n_gemv, cl);
-    if (cl > 1 && !t.cl) continue;
-    const size_t cost = split_read_bytes(t.m, t.cl ? cl : 1);
-    if (cost < best) {
-      best = cost;
-      best_cl = cl;
-    }
-  }
-  g.cta_start[1] = C;
-  set_split(a, C - (C > 2 * kOutCtas ? kOutCtas : 1), best_cl);
-  return launch_group<false>(g, a.cl ? best_cl : 1, st);
+  return launch_group<false>(g, st);
 }
 
 size_t group_ws_bytes() { return kGroupWsPartials + (size_t)kMaxCtas * kTile * 4; }
 
 cudaError_t launch_decode_group(int n, const grinqh_linear *lins, void *ws, cudaStream_t st) {
   char *w = static_cast<char *>(ws);
+  DecodeGroup g = {};
+  g.n = n;
+  // CTAs in proportion to each linear's plane bytes (tiles x d_in x P), at least one each
   const int C = device_sms();
-  bool aligned = true;
-  for (int j = 0; j < n; ++j) aligned = aligned && (lins[j].d_out / 16) % 4 == 0;
-  // CTAs in proportion to each linear's plane bytes (tiles x d_in x P), at least one
-  // cluster each, in whole clusters; the cluster size whose largest split read is smallest
-  DecodeGroup best_g = {};
-  int best_cl = 1;
-  size_t best = ~size_t(0);
-  for (int cl : {4, 2, 1}) {
-    if (C % cl != 0 || C < n * cl) continue;
-    if (cl > 1 && (aligned ? cluster_capacity<true, true>(cl) : cluster_capacity<false, true>(cl)) < C)
-      continue;
-    const int units = C / cl;  // clusters to share out
-    double tot = 0.0, wgt[kMaxGroup];
-    for (int j = 0; j < n; ++j) {
-      const int tiles = (lins[j].d_out + kTile - 1) / kTile;
-      wgt[j] = (double)tiles * lins[j].d_in * (lins[j].b_max / 2);
-      tot += wgt[j];
-    }
-    int cnt[kMaxGroup], used = 0;
-    for (int j = 0; j < n; ++j) {
-      cnt[j] = (int)((double)units * wgt[j] / tot);
-      if (cnt[j] < 1) cnt[j] = 1;
-      used += cnt[j];
-    }
-    while (used > units) {  // rounding up the small ones may overshoot: trim the largest
-      int big = 0;
-      for (int j = 1; j < n; ++j)
-        if (cnt[j] > cnt[big]) big = j;
-      --cnt[big];
-      --used;
-    }
-    DecodeGroup g = {};
-    g.n = n;
-    int tile_off = 0;
-    size_t cost = 0;
-    bool any_cl = false;
-    for (int j = 0; j < n; ++j) {
-      const grinqh_linear &l = lins[j];
-      g.cta_start[j + 1] = g.cta_start[j] + cnt[j] * cl;
-      DecodeArgs &a = g.lin[j];
-      a = make_args(l.planes, l.s, l.z, l.x, l.theta, l.phi, l.d_in, l.d_out, l.b_max, l.y);
-      set_split(a, cnt[j] * cl, cl);
-      any_cl = any_cl || a.cl;
-      a.counters = reinterpret_cast<unsigned long long *>(w + kGroupWsCounters) + tile_off;
-      a.partials = reinterpret_cast<float *>(w + kGroupWsPartials) + (size_t)g.cta_start[j] * kTile;
-      a.error = &reinterpret_cast<WsHeader *>(w)->error;
-      a.reserve_out = 0;
-      tile_off += a.tiles * (a.cl ? cl : 1);
-      const size_t cj = split_read_bytes(a.m, a.cl ? cl : 1);
-      cost = cj > cost ? cj : cost;
-    }
-    if (cl > 1 && !any_cl) continue;
-    if (cost < best) {
-      best = cost;
-      best_cl = cl;
-      best_g = g;
-    }
+  double tot = 0.0, wgt[kMaxGroup];
+  for (int j = 0; j < n; ++j) {
+    const int tiles = (lins[j].d_out + kTile - 1) / kTile;
+    wgt[j] = (double)tiles * lins[j].d_in * (lins[j].b_max / 2);
+    tot += wgt[j];
   }
-  return launch_group<true>(best_g, best_cl, st);
+  int cnt[kMaxGroup], used = 0;
+  for (int j = 0; j < n; ++j) {
+    cnt[j] = (int)((double)C * wgt[j] / tot);
+    if (cnt[j] < 1) cnt[j] = 1;
+    used += cnt[j];
+  }
+  while (used > C) {  // rounding up the small ones may overshoot: trim the largest
+    int big = 0;
+    for (int j = 1; j < n; ++j)
+      if (cnt[j] > cnt[big]) big = j;
+    --cnt[big];
+    --used;
+  }
+  int tile_off = 0;
+  for (int j = 0; j < n; ++j) {
+    const grinqh_linear &l = lins[j];
+    g.cta_start[j + 1] = g.cta_start[j] + cnt[j];
+    DecodeArgs &a = g.lin[j];
+    a = make_args(l.planes, l.s, l.z, l.x, l.theta, l.phi, l.d_in, l.d_out, l.b_max, l.y, cnt[j]);
+    a.counters = reinterpret_cast<unsigned *>(w + kGroupWsCounters) + tile_off;
+    a.partials = reinterpret_cast<float *>(w + kGroupWsPartials) + (size_t)g.cta_start[j] * kTile;
+    a.error = &reinterpret_cast<WsHeader *>(w)->error;
+    a.reserve_out = 0;
+    tile_off += a.tiles;
+  }
+  return launch_group<true>(g, st);
 }
 
 }  // namespace grinqh

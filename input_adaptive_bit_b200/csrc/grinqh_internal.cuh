@@ -24,8 +24,7 @@ constexpr int kDecodeMaxDin = 65536;            // largest d_in of the fused dec
 // Device error codes written to the workspace error word.
 constexpr int kDevErrStreamMismatch = 1;  // gemv saw a unit stream of another d_in / b_max
 constexpr int kDevErrBadUnit = 2;         // a unit record outside [0, d_in) x [0, P) (skipped)
-constexpr int kDevErrSplitKTimeout = 3;   // decode: a split-K partial was missing when its share
-                                          // was summed (a stale arrival word); see decode.cu
+constexpr int kDevErrSplitKTimeout = 3;   // decode: a split-K wait gave up (see decode.cu)
 constexpr int kDevErrPrefillTimeout = 4;  // prefill: a wait on the tensor cores gave up
 constexpr int kDevErrPipeTimeout = 5;     // decode: a wait on the copy/MMA pipeline gave up
 
@@ -192,13 +191,13 @@ cudaError_t launch_decode(const uint32_t *planes, const uint16_t *s, const uint1
                           const uint16_t *x, const float *theta, const float *phi, int d_in,
                           int d_out, int b_max, float *y, uint8_t *b, int32_t *lists,
                           int32_t *counts, float *grp_sums, void *ws, cudaStream_t st);
-// The same launch with the split-K state at explicit addresses: `counters` (64-bit
-// arrival words, zero; at least 2 ceil(d_out / 1024) of them, and at least 148),
-// `partials` (fp32, kMaxCtas x 1024) and the device error word.
+// The same launch with the split-K state at explicit addresses: `counters` (arrival
+// words, zero; at least ceil(d_out / 1024) of them), `partials` (fp32, kMaxCtas x
+// 1024) and the device error word.
 cudaError_t launch_decode_split(const uint32_t *planes, const uint16_t *s, const uint16_t *z,
                                 const uint16_t *x, const float *theta, const float *phi, int d_in,
                                 int d_out, int b_max, float *y, uint8_t *b, int32_t *lists,
-                                int32_t *counts, float *grp_sums, unsigned long long *counters,
+                                int32_t *counts, float *grp_sums, unsigned *counters,
                                 float *partials, int *error, cudaStream_t st);
 // Argument checks of grinqh_decode_gemv (everything but the workspace): GRINQH_OK
 // or the status it returns, with the message set.

@@ -19,11 +19,11 @@ namespace grinqh {
 namespace {
 
 // Scratch layout: the error word (a 256-byte header), the split-K arrival
-// words (64-bit, two per 1024-output tile: enough for d_out up to 2^24), then
-// the partial sums of up to kMaxCtas CTAs.  None of it depends on d_in, so the
+// words (one per 1024-output tile: enough for d_out up to 2^24), then the
+// partial sums of up to kMaxCtas CTAs.  None of it depends on d_in, so the
 // scratch serves every shape grinqh_decode_gemv takes.
 constexpr size_t kNaCounters = 256;
-constexpr size_t kNaPartials = kNaCounters + (size_t)2 * ((1 << 24) / 1024) * 8;
+constexpr size_t kNaPartials = kNaCounters + (size_t)((1 << 24) / 1024) * 4;
 constexpr size_t kNoAllocBytes = kNaPartials + (size_t)kMaxCtas * 1024 * 4;  // about 1.2 MB
 static_assert(kNaPartials % 256 == 0, "aligned regions");
 
@@ -75,13 +75,12 @@ extern "C" int grinqh_decode_gemv_noalloc(const uint32_t *planes, const uint16_t
   // not: the words this shape uses are cleared first.  The error word is not:
   // it keeps the first error until it is read.
   const size_t tiles = ((size_t)d_out + 1023) / 1024;
-  e = cudaMemsetAsync(sc + kNaCounters, 0, 2 * tiles * 8 > 148 * 8 ? 2 * tiles * 8 : 148 * 8,
-                      (cudaStream_t)stream);
+  e = cudaMemsetAsync(sc + kNaCounters, 0, tiles * 4, (cudaStream_t)stream);
   if (e != cudaSuccess)
     return record_error(GRINQH_ERR_CUDA, "grinqh_decode_gemv_noalloc: clearing scratch: %s",
                         cudaGetErrorString(e));
   e = launch_decode_split(planes, s, z, x, theta, phi, d_in, d_out, b_max, y, nullptr, nullptr,
-                          nullptr, nullptr, reinterpret_cast<unsigned long long *>(sc + kNaCounters),
+                          nullptr, nullptr, reinterpret_cast<unsigned *>(sc + kNaCounters),
                           reinterpret_cast<float *>(sc + kNaPartials), reinterpret_cast<int *>(sc),
                           (cudaStream_t)stream);
   if (e != cudaSuccess)

@@ -1,6 +1,5 @@
 // pipeline.cuh -- device helpers of the decode kernels (decode.cu, batch.cu):
-// cp.async and 1-D bulk copies, mbarrier waits with a bound, the m16n8k16 MMA,
-// thread-block cluster barriers and loads from a peer CTA's shared memory.
+// cp.async and 1-D bulk copies, mbarrier waits with a bound, the m16n8k16 MMA.
 #pragma once
 
 #include "grinqh_internal.cuh"
@@ -97,6 +96,11 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+__device__ __forceinline__ unsigned ld_acquire(const unsigned *p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];\n" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
 __device__ __forceinline__ unsigned long long ld_acquire64(const unsigned long long *p) {
   unsigned long long v;
   asm volatile("ld.acquire.gpu.global.u64 %0, [%1];\n" : "=l"(v) : "l"(p) : "memory");
@@ -106,30 +110,6 @@ __device__ __forceinline__ unsigned long long ld_acquire64(const unsigned long l
 // Barrier of the first n threads of the CTA only (named barrier 1).
 template <int N>
 __device__ __forceinline__ void sync_first() { asm volatile("bar.sync 1, %0;\n" ::"n"(N)); }
-
-// Thread-block cluster: barrier halves, rank, and a 16-byte load from a peer's
-// shared memory at the address of `local` in this CTA.
-__device__ __forceinline__ void cluster_arrive() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n" ::: "memory");
-}
-__device__ __forceinline__ void cluster_wait() {
-  asm volatile("barrier.cluster.wait.acquire.aligned;\n" ::: "memory");
-}
-__device__ __forceinline__ uint32_t cluster_rank() {
-  uint32_t r;
-  asm("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-__device__ __forceinline__ float4 ld_peer_f4(const float *local, uint32_t rank) {
-  uint32_t ra;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(smem_u32(local)), "r"(rank));
-  float4 v;
-  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
-               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-               : "r"(ra)
-               : "memory");
-  return v;
-}
 
 __device__ __forceinline__ float4 f4add(float4 a, float4 b) {
   return make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w);

@@ -205,7 +205,7 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_kernel(const __grid_cons
   extern __shared__ __align__(128) unsigned char smem[];
   __shared__ uint32_t s_tmem;
   __shared__ __align__(8) uint64_t s_full_p[kSP], s_empty_p[kSP], s_full_x[kSX], s_empty_x[kSX];
-  __shared__ __align__(8) uint64_t s_a_full[2], s_a_empty[2], s_acc_full, s_acc_empty;
+  __shared__ __align__(8) uint64_t s_a_full[2], s_a_empty[2], s_acc_full, s_acc_empty, s_drain;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   if (warp == kMmaWarp) {
@@ -229,6 +229,7 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_kernel(const __grid_cons
     }
     mbar_init(&s_acc_full, 1);
     mbar_init(&s_acc_empty, kBuilders);
+    mbar_init(&s_drain, 1);
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
   }
   tc_fence_before();
@@ -339,9 +340,10 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_kernel(const __grid_cons
     uint32_t ci = 0;
     for (long long u = u_lo; u < u_hi;) {
       const Piece pc = piece_at(a, u, u_hi);
-      for (int i = 0; i < pc.n; ++i, ++ci) {
+      for (int i = 0; i < pc.n && ok; ++i, ++ci) {
         const int sp = (int)(ci % kSP);
         if (ci >= kSP) wait(&s_empty_p[sp], ci / kSP - 1);
+        if (!ok) break;  // a wait gave up: issue nothing more
         const int g = pc.g0 + i;
 #pragma unroll
         for (int rr = 0; rr < 2; ++rr) {
@@ -369,9 +371,10 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_kernel(const __grid_cons
     uint32_t ci = 0;
     for (long long u = u_lo; u < u_hi;) {
       const Piece pc = piece_at(a, u, u_hi);
-      for (int i = 0; i < pc.n; ++i, ++ci) {
+      for (int i = 0; i < pc.n && ok; ++i, ++ci) {
         const int sx = (int)(ci % kSX);
         if (ci >= kSX) wait(&s_empty_x[sx], ci / kSX - 1);
+        if (!ok) break;  // a wait gave up: issue nothing more
         const int k0 = (pc.g0 + i) * kPK;
         unsigned char *dst = smem + kOffX + (size_t)sx * kXSlot + (c >> 1) * pc.n_pad * 32 + (c & 1) * 128 + tk0 * 16;
         for (int j = 0; j < pc.n_pad / 8; ++j) {
@@ -398,6 +401,7 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_kernel(const __grid_cons
         const int sx = (int)(ci % kSX);
         wait(&s_a_full[ci & 1], ci >> 1);
         wait(&s_full_x[sx], ci / kSX);
+        if (!ok) break;  // a wait gave up: issue no more MMAs
         tc_fence_after();
         const uint32_t a_addr = smem_u32(smem + kOffA + (size_t)(ci & 1) * kABuf);
         const uint32_t b_addr = smem_u32(smem + kOffX + (size_t)sx * kXSlot);
@@ -419,6 +423,16 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_kernel(const __grid_cons
     }
   }
 
+  // Before the tensor memory is freed and the CTA exits, nothing may still be in flight:
+  // every thread's own cp.async copies have landed, and the MMA lane commits once
+  // more and waits (bounded) for all of its MMAs -- on a correct run they are
+  // complete already; after a wait that gave up this is what keeps an MMA from
+  // writing tensor memory that has been freed.
+  asm volatile("cp.async.wait_all;\n" ::: "memory");
+  if (warp == kMmaWarp && lane == 0) {
+    tc_commit(&s_drain);
+    if (!mbar_wait(&s_drain, 0)) ok = false;
+  }
   tc_fence_before();
   __syncthreads();
   if (warp == kMmaWarp) {

@@ -5,6 +5,8 @@ CTAs, every split-K factor from 144 CTAs per tile down to one (with and
 without cluster sums), the optional outputs (bit-exact with grinqh_assign, or
 skipped), and a stale split-K counter reported as a device error while y
 stays right."""
+import time
+
 import numpy as np
 import pytest
 import torch
@@ -127,9 +129,9 @@ def test_large_activations_use_a_scaled_b_column():
 @pytest.mark.parametrize("d_out", [1024, 2048, 48 * 1024, 72 * 1024, 144 * 1024])
 def test_split_k_shares_every_ctas_per_tile(d_out):
     # one tile (every GEMV CTA takes a slice of the same 1024 outputs) down to one
-    # CTA per tile: the partial sums meet in cluster pairs and in global memory in a
-    # fixed order; y must be the same on a second call and the device error word
-    # must stay clear
+    # CTA per tile: each CTA of a tile waits for the others and adds its share of
+    # the partial sums; y must be the same on a second call (fixed order) and the
+    # device error word must stay clear
     from input_adaptive_bit_b200 import grinqh_check_device_error
     d_in = 512
     q, s, z, x, theta = cheap_case(8, d_in, d_out, 8)
@@ -143,31 +145,60 @@ def test_split_k_shares_every_ctas_per_tile(d_out):
     grinqh_check_device_error(lin.ws)  # raises if a split-K wait gave up
 
 
-def test_stale_arrival_count_is_reported_and_y_is_still_right():
-    # A workspace left with one stale arrival in the count of a split tile's
-    # arrival word (the call requires it zeroed): the arrival that the count
-    # takes for the last one sees from the arrival bits which partial sum is
-    # missing, waits for it, sets device error 3 and writes the right y; the
-    # word is left zeroed, so the next call reports nothing.
+def test_split_k_wait_gives_up_on_a_stale_arrival_count():
+    # A workspace left with one stale arrival on a tile's arrival word (the call
+    # requires it zeroed): the tile's count completes one arrival early, the CTAs
+    # that arrive after it wait for a count that never comes, give up after their
+    # poll limit, set device error 3 and let the kernel finish; the context stays
+    # usable, and a call on the cleared workspace is right and reports nothing.
     from input_adaptive_bit_b200 import ERR_DEVICE, GrinqhError, grinqh_check_device_error
-    # 8 tiles: 18 CTAs per tile, so at most 18 partial sums meet in any share
-    q, s, z, x, theta = cheap_case(9, 512, 8192, 8)
+    q, s, z, x, theta = cheap_case(9, 512, 1024, 8)  # one tile: every GEMV CTA shares it
     lin = GrinqhLinear(q, s, z, 8)
     xd, th = to_dev(x), to_dev(theta)
-    count = lin.ws[260:264].view(torch.int32)  # high half of tile 0's first arrival word
-    count.fill_(1)
-    y = lin.decode(xd, th, outputs=False)
+    counters = lin.ws[256:260].view(torch.int32)  # the tile's arrival word (after the header)
+    counters.fill_(1)
+    lin.decode(xd, th, outputs=False)
     torch.cuda.synchronize()
     with pytest.raises(GrinqhError) as err:
         grinqh_check_device_error(lin.ws)
     assert err.value.status == ERR_DEVICE and "code 3" in str(err.value)
-    assert not lin.ws[256:256 + 8 * 64].any()  # every arrival word is back at zero
-    b_ref = oracle.assign(x, theta, 8)
-    check_y({"y": y.cpu().numpy().astype(np.float64)}, oracle.pack(q, 8), s, z, x, b_ref, 8)
+    lin.ws.zero_()
     _, out = run_layer(None, None, None, x, theta, 8, lin=lin, path="fused")
     b_ref = check_assign(out, x, theta, 8)
     check_y(out, oracle.pack(q, 8), s, z, x, b_ref, 8)
     grinqh_check_device_error(lin.ws)
+    assert not lin.ws[256:256 + 4 * 64].any()  # every arrival word is back at zero
+
+
+def test_y_is_right_when_some_ctas_cannot_start_until_others_gave_up():
+    # Other work holds a few SMs (single-thread kernels that sleep ~0.8 s on side
+    # streams: the decode kernel's CTAs need a whole SM each, so those SMs stay shut
+    # to it).  CTAs of the same tiles that are running wait for them, give up after
+    # their poll limit (device error 3), mark the tiles' arrival words and exit; the
+    # late CTAs then run, and each tile's last arrival sees the mark and sums the
+    # whole tile.  y must still be the oracle's.
+    from input_adaptive_bit_b200 import ERR_DEVICE, GrinqhError, grinqh_check_device_error
+    q, s, z, x, theta = cheap_case(10, 1024, 4096, 8)  # 4 tiles, 36 CTAs each
+    lin = GrinqhLinear(q, s, z, 8)
+    xd, th = to_dev(x), to_dev(theta)
+    y = torch.full((4096,), float("nan"), dtype=torch.float32, device="cuda")
+    torch.cuda.synchronize()
+    side = [torch.cuda.Stream() for _ in range(4)]
+    for st in side:
+        with torch.cuda.stream(st):
+            torch.cuda._sleep(int(0.8 * 1.9e9))  # ~0.8 s of clock cycles, one thread
+    time.sleep(0.05)  # the sleepers are resident first
+    main = torch.cuda.Stream()
+    with torch.cuda.stream(main):
+        lin.decode(xd, th, y=y, outputs=False, stream=main)
+    torch.cuda.synchronize()
+    b_ref = oracle.assign(x, theta, 8)
+    check_y({"y": y.cpu().numpy().astype(np.float64)}, oracle.pack(q, 8), s, z, x, b_ref, 8)
+    try:
+        grinqh_check_device_error(lin.ws)  # 3 if a wait gave up (expected, not required)
+    except GrinqhError as err:
+        assert err.value.status == ERR_DEVICE and "code 3" in str(err.value)
+    assert not lin.ws[256:256 + 4 * 64].any()  # every arrival word is back at zero
 
 
 @pytest.mark.parametrize("shapes", [
