@@ -361,8 +361,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
   }
   if (c >= C_eff) return;
 
-  for (int q = tid; q < kTile; q += kThreads) s_red[q] = 0.0f;  // (the first window's barrier orders it)
-
   int *s_ccnt = reinterpret_cast<int *>(smem + kSmChunkCnt);
   float4 *s_wsum = reinterpret_cast<float4 *>(smem + kSmWarpSum);
   uint4 *s_wbal = reinterpret_cast<uint4 *>(smem + kSmWarpBal);
@@ -684,23 +682,20 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     }
     const int ol = 128 * ob + 16 * fg + 8 * (tq & 1) + 4 * (tq >> 1);  // first of 4 outputs
     const int obase = tile * kTile;
-    // the two k-parity warps of a block add into s_red (zero here): a sum of two values
-    // does not depend on their order, so the CTA's partial is deterministic
-#pragma unroll
-    for (int i = 0; i < 4; ++i) atomicAdd(s_red + ol + i, fin[i]);
+    // odd-k warps hand their sums to the even-k warp of the same block
+    __syncthreads();  // s_red of the previous tile is consumed
+    if (kp == 1) *reinterpret_cast<float4 *>(s_red + ol) = make_float4(fin[0], fin[1], fin[2], fin[3]);
     __syncthreads();
+    if (kp == 0) {
+      const float4 o = *reinterpret_cast<const float4 *>(s_red + ol);
+      fin[0] += o.x;
+      fin[1] += o.y;
+      fin[2] += o.z;
+      fin[3] += o.w;
+    }
     if (m == 1) {  // the whole tile's rows: y directly
-      for (int q = tid; q < kTile / 4; q += kThreads) {
-        const float4 v = reinterpret_cast<const float4 *>(s_red)[q];
-        reinterpret_cast<float4 *>(s_red)[q] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);  // for the next tile
-        const int o = obase + 4 * q;  // d_out % 16 == 0: a float4 is wholly in or out
-        if (o < a.d_out) {
-          a.y[o] = v.x;
-          a.y[o + 1] = v.y;
-          a.y[o + 2] = v.z;
-          a.y[o + 3] = v.w;
-        }
-      }
+      if (kp == 0 && obase + ol < a.d_out)  // d_out % 16 == 0: the 4 outputs are wholly in or out
+        for (int i = 0; i < 4; ++i) a.y[obase + ol + i] = fin[i];
       continue;
     }
     // ---- split-K: the m partial tiles of a tile meet in global memory.  Every CTA
@@ -713,20 +708,22 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     // own arrival returns, then sums the whole tile itself.  So every output is
     // written, by its owner or by the last arrival (the same bits either way). ----
     const int c_first = (c / m) * m;
-    if (tid < kTile / 4)
-      reinterpret_cast<float4 *>(a.partials + (size_t)c * kTile)[tid] =
-          reinterpret_cast<const float4 *>(s_red)[tid];
+    if (kp == 0)
+      *reinterpret_cast<float4 *>(a.partials + (size_t)c * kTile + ol) =
+          make_float4(fin[0], fin[1], fin[2], fin[3]);
     __syncthreads();
     if (tid == 0) {
       unsigned *word = a.counters + tile;
-      asm volatile("fence.sc.gpu;\n" ::: "memory");  // the partial (ordered before by the barrier)
-      const unsigned old = atomicAdd(word, 1u);
+      asm volatile("fence.acq_rel.gpu;\n" ::: "memory");  // the partial (ordered before by the
+                                                             // barrier), then the arrival
+      const unsigned old = atom_add_acq_rel(word, 1u);
       const unsigned cnt = old & kCountMask;
       int role;  // 0: sum the own share, 1: sum the whole tile, 2: gave up
-      if (cnt == (unsigned)(m - 1)) {  // the last arrival: bring the count back to zero
+      if (cnt == (unsigned)(m - 1)) {
+        // the last arrival: the count reads m now (the waiters' signal); bring it back to
+        // zero for the next launch, and clear a mark it has acted on
         role = (old & kGaveUp) ? 1 : 0;
-        atomicSub(word, (unsigned)m);
-        if (role == 1) atomicAnd(word, ~kGaveUp);
+        red_add(word, role == 1 ? (unsigned)(-m) - kGaveUp : (unsigned)(-m));
       } else {
         // complete once the count reads m (the last arrival) or 0 (reset after it)
         role = 2;
@@ -741,39 +738,55 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         if (role == 2) {
           // mark the word, then look once more: either the last arrival has come (and the
           // mark is stale but harmless), or it has not and will see the mark
-          asm volatile("fence.sc.gpu;\n" ::: "memory");
-          const unsigned c2 = atomicOr(word, kGaveUp) & kCountMask;
+          const unsigned c2 = atom_or_acq_rel(word, kGaveUp) & kCountMask;
           if (c2 == 0u || c2 == (unsigned)m) role = 0;
           else atomicCAS(a.error, 0, kDevErrSplitKTimeout);
         }
       }
-      asm volatile("fence.sc.gpu;\n" ::: "memory");  // the others' partials are visible
       s_misc[1] = role;
     }
     __syncthreads();
     const int role = s_misc[1];
-    if (role != 2) {
-      // the quads [Q k / m, Q (k + 1) / m) of share k, Q = kTile / 4: share `part`, or all
-      const int q0 = role == 1 ? 0 : (kTile / 4) * part / m;
-      const int nq = role == 1 ? kTile / 4 : (kTile / 4) * (part + 1) / m - q0;
-      float4 *stage = reinterpret_cast<float4 *>(smem);  // [parts][nq]: the idle ring
-      const int per_pass = nq == kTile / 4 ? kFixParts : m;
-      float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-      for (int k0 = 0; k0 < m; k0 += per_pass) {
-        const int np = min(per_pass, m - k0);
-        for (int q = tid; q < np * nq; q += kThreads) {
-          const int k = q / nq, qq = q - k * nq;
-          cp_async16(stage + q, a.partials + (size_t)(c_first + k0 + k) * kTile + 4 * (q0 + qq), 16);
+    if (role == 0) {
+      // this CTA's share: quads [Q part / m, Q (part + 1) / m) of the tile's Q = kTile / 4;
+      // m <= kMaxCtas <= Q, so every share is non-empty, and m nq <= Q + m <= kThreads
+      static_assert(kMaxCtas <= kTile / 4 && kTile / 4 + kMaxCtas <= kThreads, "split-K shares");
+      const int q0 = (kTile / 4) * part / m, nq = (kTile / 4) * (part + 1) / m - q0;
+      float4 *s_fix = reinterpret_cast<float4 *>(smem + kSmRing);  // [m][nq]; the ring is idle
+      for (int t = tid; t < m * nq; t += kThreads) {
+        const int cc = t / nq, qq = t - cc * nq;
+        s_fix[t] = __ldcg(reinterpret_cast<const float4 *>(a.partials + (size_t)(c_first + cc) * kTile) +
+                          q0 + qq);
+      }
+      __syncthreads();
+      if (tid < nq) {
+        float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        for (int cc = 0; cc < m; ++cc) acc = f4add(acc, s_fix[cc * nq + tid]);  // in CTA order
+        const int o = obase + 4 * (q0 + tid);
+        if (o < a.d_out) {
+          a.y[o] = acc.x;
+          a.y[o + 1] = acc.y;
+          a.y[o + 2] = acc.z;
+          a.y[o + 3] = acc.w;
         }
-        cp_async_commit();
-        cp_async_wait<0>();
+      }
+    } else if (role == 1) {
+      // the whole tile (a CTA of it gave up waiting): every share, in the same order
+      float4 *stage = reinterpret_cast<float4 *>(smem);  // [kFixParts][kTile / 4]: the idle ring
+      float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+      for (int k0 = 0; k0 < m; k0 += kFixParts) {
+        const int np = min(kFixParts, m - k0);
+        for (int q = tid; q < np * (kTile / 4); q += kThreads) {
+          const int k = q / (kTile / 4), o4 = q % (kTile / 4);
+          stage[q] = __ldcg(reinterpret_cast<const float4 *>(a.partials + (size_t)(c_first + k0 + k) * kTile) + o4);
+        }
         __syncthreads();
-        if (tid < nq)
-          for (int k = 0; k < np; ++k) acc = f4add(acc, stage[k * nq + tid]);  // in CTA order
+        if (tid < kTile / 4)
+          for (int k = 0; k < np; ++k) acc = f4add(acc, stage[k * (kTile / 4) + tid]);
         __syncthreads();
       }
-      const int o = obase + 4 * (q0 + tid);
-      if (tid < nq && o < a.d_out) {
+      const int o = obase + 4 * tid;
+      if (tid < kTile / 4 && o < a.d_out) {
         a.y[o] = acc.x;
         a.y[o + 1] = acc.y;
         a.y[o + 2] = acc.z;
