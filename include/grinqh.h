@@ -62,7 +62,8 @@ const char *grinqh_last_error(void);
  * workspace carries the compacted unit stream from assign to gemv, the
  * split-K partial sums, the split-K arrival counters and a device error word.
  * It MUST be zero-filled once after allocation (e.g. cudaMemsetAsync); every
- * call leaves the counters and the error word back at zero.  One workspace
+ * call leaves its split-K state (counters, and the fused decode's partial
+ * words) and the error word back at zero.  One workspace
  * may serve several layers in sequence on one stream (size it for the
  * largest), but calls that overlap in time need distinct workspaces. */
 size_t grinqh_workspace_bytes(int d_in, int d_out, int b_max);
@@ -143,15 +144,16 @@ int grinqh_gemv(const uint32_t *planes, const uint16_t *s, const uint16_t *z,
  * the wait, and every output is written after it.  So theta and phi must not
  * be written by the kernel launched immediately before this call on the same
  * stream (a copy, an event or any other kernel in between lifts this).
- * Device errors (grinqh_check_device_error): 3 if a split-K share was about to
- * be summed with a partial sum missing, which happens only when the
- * workspace's arrival words were not left zeroed (where a share has at most 32
- * partial sums the call sees who is missing, waits for them, writes the right
- * y and leaves the word zeroed); 5 if a wait inside the
- * kernel's copy/MMA pipeline gave up (about a second; never on a correct
- * launch), in which case y is not valid.  No CTA waits for another CTA outside
- * its thread-block cluster, so the result does not depend on how many of the
- * launch's CTAs the GPU runs at the same time. */
+ * Launch: cooperative (every CTA is resident at once; the launch waits for room
+ * on the GPU, and fails with GRINQH_ERR_CUDA if the grid cannot fit, e.g. under
+ * an SM-limited MPS client), so the split-K waits between the CTAs of one output
+ * tile always end, whatever else the GPU runs.
+ * Device errors (grinqh_check_device_error): 3 if a split-K wait gave up (about
+ * half a second; never on a correct launch) or a split-K partial word of the
+ * workspace was not zero when the call started (the workspace was not left
+ * zeroed: after any device error, let grinqh_check_device_error clear it); 5 if
+ * a wait inside the kernel's copy/MMA pipeline gave up (about a second; never on
+ * a correct launch).  In both cases y is not valid. */
 int grinqh_decode_gemv(const uint32_t *planes, const uint16_t *s, const uint16_t *z,
                        const uint16_t *x, const float *theta, const float *phi, int d_in,
                        int d_out, int b_max, float *y, uint8_t *b, int32_t *lists,
@@ -243,7 +245,8 @@ int grinqh_prefill_gemm(const uint32_t *planes, const uint16_t *s, const uint16_
 
 /* Reads and clears the device error word of `ws` (synchronises `stream`).
  * Returns GRINQH_OK, or GRINQH_ERR_DEVICE with the device code in
- * grinqh_last_error(). */
+ * grinqh_last_error(); in that case it also zeroes the workspace's split-K
+ * state (its fixed-offset part), which a failed call may have left behind. */
 int grinqh_check_device_error(void *ws, void *stream);
 
 /* ---- Dense 4-bit comparator (not a GRINQH step) ------------------------------
@@ -265,8 +268,8 @@ int grinqh_gemv_dense4(const uint32_t *w4, const uint16_t *s, const uint16_t *z,
  * every byte of device memory and only hands its plug-ins streams and tensors,
  * or a latency-critical path that must never enter the allocator.  It runs
  * the fused decode kernel (grinqh_decode_gemv without its optional outputs),
- * keeping its split-K state (partial sums and arrival words) and its device
- * error word in a fixed array of about 1.2 MB that the library reserves
+ * keeping its split-K partial sums and its device error word in a fixed
+ * array of about 1 MB that the library reserves
  * on every GPU that loads it and holds until exit; it calls no
  * cudaMalloc/cudaFree.
  *   planes, s, z  the packed layer (as for grinqh_gemv); x, theta, phi as for
@@ -276,11 +279,11 @@ int grinqh_gemv_dense4(const uint32_t *w4, const uint16_t *s, const uint16_t *z,
  *   failed call.  The array holds the split-K state of every accepted shape.
  * The first call on each device looks up the array's device address
  * (cudaGetSymbolAddress) with that device current; make that first call
- * before any stream capture.  Every call shares the one array and leaves its
- * contents behind: each call first clears the arrival words it uses (one
- * cudaMemsetAsync on `stream`), so calls that overlap on the GPU --
- * several streams, or several host threads on one device -- race and must be
- * serialised by the caller.  The device error word is not cleared by a call:
+ * before any stream capture.  Every call shares the one array (a completed
+ * call leaves its split-K words at zero; a call is one kernel launch and
+ * nothing else), so calls that overlap on the GPU -- several streams, or
+ * several host threads on one device -- race and must be serialised by the
+ * caller.  The device error word is not cleared by a call:
  * it keeps the first device error (codes as for grinqh_decode_gemv) until
  * grinqh_noalloc_check_device_error reads it. */
 int grinqh_decode_gemv_noalloc(const uint32_t *planes, const uint16_t *s, const uint16_t *z,

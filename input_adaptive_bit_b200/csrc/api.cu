@@ -311,7 +311,11 @@ int grinqh_check_device_error(void *ws, void *stream) {
   const int zero = 0;
   cudaStream_t st = (cudaStream_t)stream;
   cudaError_t e = cudaMemcpyAsync(&code, ws, sizeof code, cudaMemcpyDeviceToHost, st);
-  if (e == cudaSuccess) e = cudaMemcpyAsync(ws, &zero, sizeof zero, cudaMemcpyHostToDevice, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e == cudaSuccess)
+    e = code == 0 ? cudaMemcpyAsync(ws, &zero, sizeof zero, cudaMemcpyHostToDevice, st)
+                  // a failed call may have left split-K state: clear the fixed-offset part
+                  : cudaMemsetAsync(ws, 0, grinqh::ws_fixed_end(), st);
   if (e == cudaSuccess) e = cudaStreamSynchronize(st);
   TRY(cuda_status(e, "grinqh_check_device_error"));
   if (code != 0) return fail(GRINQH_ERR_DEVICE, "device error code %d", code);

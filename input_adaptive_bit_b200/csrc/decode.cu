@@ -53,7 +53,7 @@ using namespace pipe;
 constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
 constexpr int kBlocks = 8;            // 128-output blocks of a tile; warps w and w + 8 share one
-constexpr int kTile = 1024;           // outputs per CTA tile (8 blocks x 128)
+constexpr int kTile = kDecodeTileOut;  // outputs per CTA tile (8 blocks x 128)
 constexpr int kTileW = kTile / 16;    // 64 words = 256 bytes per unit and tile
 constexpr int kRow = kTileW + 4;      // shared words per unit row: conflict-free fragment loads
 constexpr int kK = 16;                // units per MMA k-step
@@ -66,17 +66,13 @@ constexpr int kMaxG = kDecodeMaxDin / kGroup;
 constexpr int kXCache = 16384;        // rows of x held in shared memory
 constexpr int kGT = 16;               // output CTAs: threads per group, one 8-row chunk each
 constexpr int kChunkRows = 32;        // GEMV front end: rows per warp chunk, one per lane
-constexpr int kSpinLimit = 1 << 20;   // polls of a split-K arrival word before giving up (~0.3 s)
-constexpr int kFixParts = 40;         // whole partial tiles staged per pass of a full-tile sum
-constexpr unsigned kCountMask = 0xffffu;   // arrival word: the count of arrived CTAs ...
-constexpr unsigned kGaveUp = 1u << 31;     // ... and the mark of a CTA that stopped waiting
+constexpr int kSpinLimit = 1 << 20;   // polls of a split-K partial word before giving up (~0.5 s)
 constexpr int kOutCtas = 4;           // CTAs that write the optional outputs
 constexpr int kMaxGroup = GRINQH_MAX_GROUP;  // linears of one grouped launch
 
-// workspace of a grouped launch: the header, the arrival words of every linear's
-// tiles (fixed offset), then the partial tiles of every CTA
-constexpr size_t kGroupWsCounters = sizeof(WsHeader);
-constexpr size_t kGroupWsPartials = (kGroupWsCounters + (size_t)kMaxTiles * 4 + 255) & ~size_t(255);
+// workspace of a grouped launch: the header (error word), then the partial tiles of
+// every CTA (tagged words, zero between launches)
+constexpr size_t kGroupWsPartials = (sizeof(WsHeader) + 255) & ~size_t(255);
 
 // shared memory map (bytes)
 constexpr size_t kStageBytes = (size_t)kStage * kRow * 4;
@@ -95,14 +91,15 @@ constexpr size_t kSmChunkCnt = kSmRed + (size_t)kTile * 4;                  // i
 constexpr size_t kSmWarpSum = kSmChunkCnt + kSlots * 4 * 4 * 4;             // float4 [kWarps]: X, Phi, max|x|
 constexpr size_t kSmWarpBal = kSmWarpSum + kWarps * 16;                     // u32 [kWarps][2][4]: ballots
 constexpr size_t kSmWarpOff = kSmWarpBal + kWarps * 32;                     // i32 [kWarps][2][4]: first units
-constexpr size_t kSmMisc = kSmWarpOff + kWarps * 32;                        // i32 [4]: the last-arrival flag
-constexpr size_t kSmBytes = kSmMisc + 16;
+constexpr size_t kSmBytes = kSmWarpOff + kWarps * 32;
 // the output CTAs keep their counts and scans where the GEMV CTAs have the ring
 constexpr size_t kSmCnt = kSmRing;                                          // u32 [kMaxG]: plane counts, bytes
 constexpr size_t kSmLoff = kSmCnt + (size_t)kMaxG * 4;                      // int4 [kMaxG]: list offsets
 constexpr size_t kSmWsum = kSmLoff + (size_t)kMaxG * 16;                    // int4 [kWarps]
 static_assert(kSmBytes <= 227 * 1024, "shared memory");
-static_assert((size_t)kFixParts * kTile * 4 <= kSmS, "the split-K staging fits below the s/z rows");
+static_assert((size_t)(kTile / 4 + kMaxCtas) * 16 <= kSmS, "the split-K staging fits below the s/z rows");
+static_assert(kTile / 4 + kMaxCtas <= 2 * (kThreads - 32), "split-K: at most two share elements per poller");
+static_assert(kTile == kBlocks * 128, "a tile is 8 blocks of 128 outputs");
 static_assert((size_t)kXCache * 2 <= (size_t)(kRing - kXSlot) * kStageBytes, "x cache fits");
 static_assert(kSmWsum + kWarps * 16 <= kSmX, "output-CTA arrays below the x cache");
 static_assert(kSmRing % 16 == 0 && kSmX % 16 == 0 && kSmS % 16 == 0 && kSmZ % 16 == 0 &&
@@ -135,8 +132,7 @@ struct DecodeArgs {
   int32_t *lists;
   int32_t *counts;
   float *grp_sums;
-  unsigned *counters;  // arrival words (count | gave-up mark), left zero by every launch
-  float *partials;    // [CTAs of this linear][kTile]
+  float *partials;    // [CTAs of this linear][kTile] tagged words, zero between launches
   int *error;         // the workspace's device error word
   int m;              // CTAs per tile (1: each CTA takes whole tiles in turn)
   int reserve_out;    // set aside the output CTAs (the single call does, whether or not
@@ -287,7 +283,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
   uint16_t *z_st = reinterpret_cast<uint16_t *>(smem + kSmZ);
   SlotInfo *s_slot = reinterpret_cast<SlotInfo *>(smem + kSmSlot);
   float *s_red = reinterpret_cast<float *>(smem + kSmRed);
-  int *s_misc = reinterpret_cast<int *>(smem + kSmMisc);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int fg = lane >> 2, tq = lane & 3;  // MMA fragment row group and column pair
@@ -352,6 +347,24 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
   asm volatile("griddepcontrol.wait;\n" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
 
+  // the first window's x (the lane's two rows): the loads go out before anything
+  // else, and the thresholds are sorted while they are in flight
+  uint32_t xr_first = 0u, inb_first = 0u;
+  if (c < C_eff && c < C_g) {
+    const int slot = warp >> 1, cc0 = 2 * (warp & 1);
+    if (slot < window_groups(g_first)) {
+      const int row0 = (g_first + slot) * kGroup + kChunkRows * cc0 + lane;
+#pragma unroll
+      for (int ci = 0; ci < 2; ++ci) {
+        const int row = row0 + kChunkRows * ci;
+        if (row >= row_lo && row < row_hi) {
+          xr_first |= (uint32_t)__ldg(a.x + row) << (16 * ci);
+          inb_first |= 1u << ci;
+        }
+      }
+    }
+  }
+
   __half2 t2[4];
   sort_thresholds(th_raw, t2);
 
@@ -387,7 +400,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
       const int row0 = (g_w + slot) * kGroup + kChunkRows * cc0 + lane;  // the lane's row in chunk cc0
       uint32_t xr = 0u, inb = 0u;  // the lane's two x values (fp16 pair) and which are in the slice
       uint32_t bal[2][4] = {{0u, 0u, 0u, 0u}, {0u, 0u, 0u, 0u}};
-      if (live) {
+      if (g_w == g_first && tile == tile_first) {
+        xr = xr_first;
+        inb = inb_first;
+      } else if (live) {
 #pragma unroll
         for (int ci = 0; ci < 2; ++ci) {
           const int row = row0 + kChunkRows * ci;
@@ -699,100 +715,78 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
       continue;
     }
     // ---- split-K: the m partial tiles of a tile meet in global memory.  Every CTA
-    // publishes its partial and counts its arrival on the tile's arrival word; once
-    // all m have arrived, every CTA adds up its own 1/m share of the outputs over the
-    // m partials in CTA order (deterministic), so the sum is spread over the tile's
-    // CTAs.  Waiting for the others needs them to be running; if one is not (the GPU
-    // is shared with other work), a waiter gives up after a bound, marks the word,
-    // and exits -- and the tile's last arrival, which sees that mark in the value its
-    // own arrival returns, then sums the whole tile itself.  So every output is
-    // written, by its owner or by the last arrival (the same bits either way). ----
+    // publishes its partial as tagged words (never zero; see tag_word), then adds up
+    // its own 1/m share of the tile's outputs over the m partials in CTA order
+    // (deterministic), polling each word until it is non-zero, and sets the words it
+    // consumed back to zero for the next launch.  The data are their own flags: no
+    // fence or counter sits between the last partial and its readers.  The launch is
+    // cooperative, so every CTA of the tile is resident and every wait ends; the poll
+    // bound only guards against a broken launch. ----
     const int c_first = (c / m) * m;
-    if (kp == 0)
-      *reinterpret_cast<float4 *>(a.partials + (size_t)c * kTile + ol) =
-          make_float4(fin[0], fin[1], fin[2], fin[3]);
-    __syncthreads();
-    if (tid == 0) {
-      unsigned *word = a.counters + tile;
-      asm volatile("fence.acq_rel.gpu;\n" ::: "memory");  // the partial (ordered before by the
-                                                             // barrier), then the arrival
-      const unsigned old = atom_add_acq_rel(word, 1u);
-      const unsigned cnt = old & kCountMask;
-      int role;  // 0: sum the own share, 1: sum the whole tile, 2: gave up
-      if (cnt == (unsigned)(m - 1)) {
-        // the last arrival: the count reads m now (the waiters' signal); bring it back to
-        // zero for the next launch, and clear a mark it has acted on
-        role = (old & kGaveUp) ? 1 : 0;
-        red_add(word, role == 1 ? (unsigned)(-m) - kGaveUp : (unsigned)(-m));
+    uint32_t *part_w = reinterpret_cast<uint32_t *>(a.partials);
+    uint32_t canary = 0u;
+    if (kp == 0) {
+      uint32_t *dst = part_w + (size_t)c * kTile + ol;
+      const uint4 t = make_uint4(tag_word(fin[0]), tag_word(fin[1]), tag_word(fin[2]), tag_word(fin[3]));
+      if (ol == 0) {
+        // the partial's first word must still be zero from the last launch: a workspace
+        // that was not left zeroed shows up here (checked after the share is summed)
+        canary = atomicExch(dst, t.x);
+        st_relaxed_u32(dst + 1, t.y);
+        st_relaxed_u32(dst + 2, t.z);
+        st_relaxed_u32(dst + 3, t.w);
       } else {
-        // complete once the count reads m (the last arrival) or 0 (reset after it)
-        role = 2;
-        for (int polls = 0; polls < kSpinLimit; ++polls) {
-          const unsigned c2 = ld_acquire(word) & kCountMask;
-          if (c2 == 0u || c2 == (unsigned)m) {
-            role = 0;
+        st_relaxed_v4(dst, t);
+      }
+    }
+    // this CTA's share: quads [Q part / m, Q (part + 1) / m) of the tile's Q = kTile / 4;
+    // m <= kMaxCtas <= Q, so every share is non-empty, and m nq <= Q + m
+    static_assert(kMaxCtas <= kTile / 4, "split-K shares");
+    const int q0 = (kTile / 4) * part / m, nq = (kTile / 4) * (part + 1) / m - q0;
+    float4 *s_fix = reinterpret_cast<float4 *>(smem + kSmRing);  // [m][nq]; the ring is idle
+    // pollers: threads 32 and up (warp 0 holds the canary's exchange), element e of
+    // the share (partial e / nq, quad e mod nq) on thread 32 + e mod (kThreads - 32)
+    const int pt = tid - 32;
+    auto elem = [&](int e) -> uint32_t * {
+      const int cc = e / nq, qq = e - cc * nq;
+      return part_w + (size_t)(c_first + cc) * kTile + 4 * (q0 + qq);
+    };
+    int gave_up = 0;
+    if (pt >= 0) {
+      for (int e = pt; e < m * nq && !gave_up; e += kThreads - 32) {
+        const uint32_t *src = elem(e);
+        uint4 v;
+        for (int polls = 0;; ++polls) {
+          v = ld_relaxed_v4(src);
+          if (v.x != 0u && v.y != 0u && v.z != 0u && v.w != 0u) break;
+          if (polls == kSpinLimit) {
+            gave_up = 1;
             break;
           }
-          __nanosleep(32);
+          __nanosleep(20);
         }
-        if (role == 2) {
-          // mark the word, then look once more: either the last arrival has come (and the
-          // mark is stale but harmless), or it has not and will see the mark
-          const unsigned c2 = atom_or_acq_rel(word, kGaveUp) & kCountMask;
-          if (c2 == 0u || c2 == (unsigned)m) role = 0;
-          else atomicCAS(a.error, 0, kDevErrSplitKTimeout);
-        }
+        s_fix[e] = make_float4(__uint_as_float(v.x), __uint_as_float(v.y), __uint_as_float(v.z),
+                               __uint_as_float(v.w));
       }
-      s_misc[1] = role;
     }
-    __syncthreads();
-    const int role = s_misc[1];
-    if (role == 0) {
-      // this CTA's share: quads [Q part / m, Q (part + 1) / m) of the tile's Q = kTile / 4;
-      // m <= kMaxCtas <= Q, so every share is non-empty, and m nq <= Q + m <= kThreads
-      static_assert(kMaxCtas <= kTile / 4 && kTile / 4 + kMaxCtas <= kThreads, "split-K shares");
-      const int q0 = (kTile / 4) * part / m, nq = (kTile / 4) * (part + 1) / m - q0;
-      float4 *s_fix = reinterpret_cast<float4 *>(smem + kSmRing);  // [m][nq]; the ring is idle
-      for (int t = tid; t < m * nq; t += kThreads) {
-        const int cc = t / nq, qq = t - cc * nq;
-        s_fix[t] = __ldcg(reinterpret_cast<const float4 *>(a.partials + (size_t)(c_first + cc) * kTile) +
-                          q0 + qq);
-      }
-      __syncthreads();
-      if (tid < nq) {
-        float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-        for (int cc = 0; cc < m; ++cc) acc = f4add(acc, s_fix[cc * nq + tid]);  // in CTA order
-        const int o = obase + 4 * (q0 + tid);
-        if (o < a.d_out) {
-          a.y[o] = acc.x;
-          a.y[o + 1] = acc.y;
-          a.y[o + 2] = acc.z;
-          a.y[o + 3] = acc.w;
-        }
-      }
-    } else if (role == 1) {
-      // the whole tile (a CTA of it gave up waiting): every share, in the same order
-      float4 *stage = reinterpret_cast<float4 *>(smem);  // [kFixParts][kTile / 4]: the idle ring
+    if (__syncthreads_or(gave_up)) {
+      if (tid == 0) atomicCAS(a.error, 0, kDevErrSplitKTimeout);
+      continue;  // y of this share is not written; the words stay for the error path
+    }
+    if (pt >= 0)
+      for (int e = pt; e < m * nq; e += kThreads - 32) st_relaxed_v4(elem(e), make_uint4(0u, 0u, 0u, 0u));  // consumed
+    if (pt >= 0 && pt < nq) {
       float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-      for (int k0 = 0; k0 < m; k0 += kFixParts) {
-        const int np = min(kFixParts, m - k0);
-        for (int q = tid; q < np * (kTile / 4); q += kThreads) {
-          const int k = q / (kTile / 4), o4 = q % (kTile / 4);
-          stage[q] = __ldcg(reinterpret_cast<const float4 *>(a.partials + (size_t)(c_first + k0 + k) * kTile) + o4);
-        }
-        __syncthreads();
-        if (tid < kTile / 4)
-          for (int k = 0; k < np; ++k) acc = f4add(acc, stage[k * (kTile / 4) + tid]);
-        __syncthreads();
-      }
-      const int o = obase + 4 * tid;
-      if (tid < kTile / 4 && o < a.d_out) {
+      for (int cc = 0; cc < m; ++cc) acc = f4add(acc, s_fix[cc * nq + pt]);  // in CTA order
+      const int o = obase + 4 * (q0 + pt);
+      if (o < a.d_out) {
         a.y[o] = acc.x;
         a.y[o + 1] = acc.y;
         a.y[o + 2] = acc.z;
         a.y[o + 3] = acc.w;
       }
     }
+    if (canary != 0u) atomicCAS(a.error, 0, kDevErrSplitKTimeout);
   }
 }
 
@@ -817,11 +811,15 @@ cudaError_t launch_variant(const DecodeGroup &g, cudaStream_t st) {
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = kSmBytes;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  // programmatic dependent launch, and cooperative: every CTA is resident at once, so
+  // the split-K waits on the other CTAs of a tile always end
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeCooperative;
+  attr[1].val.cooperative = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, decode_kernel<ALIGNED, GROUPED>, g);
 }
 
@@ -865,16 +863,15 @@ cudaError_t launch_decode(const uint32_t *planes, const uint16_t *s, const uint1
   const WsLayout L = ws_layout(d_in, d_out, b_max);
   char *w = static_cast<char *>(ws);
   return launch_decode_split(planes, s, z, x, theta, phi, d_in, d_out, b_max, y, b, lists, counts,
-                             grp_sums, reinterpret_cast<unsigned *>(w + L.counters),
-                             reinterpret_cast<float *>(w + L.partials),
+                             grp_sums, reinterpret_cast<float *>(w + L.dpartials),
                              &reinterpret_cast<WsHeader *>(w)->error, st);
 }
 
 cudaError_t launch_decode_split(const uint32_t *planes, const uint16_t *s, const uint16_t *z,
                                 const uint16_t *x, const float *theta, const float *phi, int d_in,
                                 int d_out, int b_max, float *y, uint8_t *b, int32_t *lists,
-                                int32_t *counts, float *grp_sums, unsigned *counters,
-                                float *partials, int *error, cudaStream_t st) {
+                                int32_t *counts, float *grp_sums, float *partials, int *error,
+                                cudaStream_t st) {
   DecodeGroup g = {};
   g.n = 1;
   g.cta_start[0] = 0;
@@ -887,7 +884,6 @@ cudaError_t launch_decode_split(const uint32_t *planes, const uint16_t *s, const
   a.lists = lists;
   a.counts = counts;
   a.grp_sums = grp_sums;
-  a.counters = counters;
   a.partials = partials;
   a.error = error;
   a.reserve_out = 1;
@@ -921,17 +917,14 @@ cudaError_t launch_decode_group(int n, const grinqh_linear *lins, void *ws, cuda
     --cnt[big];
     --used;
   }
-  int tile_off = 0;
   for (int j = 0; j < n; ++j) {
     const grinqh_linear &l = lins[j];
     g.cta_start[j + 1] = g.cta_start[j] + cnt[j];
     DecodeArgs &a = g.lin[j];
     a = make_args(l.planes, l.s, l.z, l.x, l.theta, l.phi, l.d_in, l.d_out, l.b_max, l.y, cnt[j]);
-    a.counters = reinterpret_cast<unsigned *>(w + kGroupWsCounters) + tile_off;
     a.partials = reinterpret_cast<float *>(w + kGroupWsPartials) + (size_t)g.cta_start[j] * kTile;
     a.error = &reinterpret_cast<WsHeader *>(w)->error;
     a.reserve_out = 0;
-    tile_off += a.tiles;
   }
   return launch_group<true>(g, st);
 }

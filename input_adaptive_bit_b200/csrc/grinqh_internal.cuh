@@ -19,12 +19,14 @@ constexpr int kMaxCtaUnits = 8192;     // bound on units per gemv CTA (sets the 
 constexpr int kNumSMs = 148;
 constexpr int kMaxTiles = (1 << 24) / kTileOut;  // d_out <= 2^24
 constexpr int kMaxCtas = 256;                   // gemv grid: one CTA per SM, at most this many
+constexpr int kDecodeTileOut = 1024;            // outputs per tile of the fused decode kernel
 constexpr int kDecodeMaxDin = 65536;            // largest d_in of the fused decode kernel
 
 // Device error codes written to the workspace error word.
 constexpr int kDevErrStreamMismatch = 1;  // gemv saw a unit stream of another d_in / b_max
 constexpr int kDevErrBadUnit = 2;         // a unit record outside [0, d_in) x [0, P) (skipped)
-constexpr int kDevErrSplitKTimeout = 3;   // decode: a split-K wait gave up (see decode.cu)
+constexpr int kDevErrSplitKTimeout = 3;   // decode: a split-K wait gave up, or a partial word
+                                          // was not zero before the launch (see decode.cu)
 constexpr int kDevErrPrefillTimeout = 4;  // prefill: a wait on the tensor cores gave up
 constexpr int kDevErrPipeTimeout = 5;     // decode: a wait on the copy/MMA pipeline gave up
 
@@ -40,11 +42,15 @@ static_assert(sizeof(WsHeader) == 256, "header size");
 
 inline __host__ __device__ size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
-// Workspace layout.  The header and the split-K counters sit at fixed offsets
-// for every shape, so one workspace can serve layers of different shapes in
-// turn: the counters return to zero after every gemv, whatever its shape.
+// Workspace layout.  The header, the split-K counters of grinqh_gemv and the
+// split-K partial words of the fused decode sit at fixed offsets for every
+// shape, so one workspace can serve layers of different shapes in turn: the
+// counters and the decode's partial words return to zero after every call,
+// whatever its shape.
 struct WsLayout {
   size_t counters;    // uint32 [kMaxTiles]: split-K arrival counters (fixed offset)
+  size_t dpartials;   // u32 [kMaxCtas][kDecodeTileOut]: the fused decode's tagged partial
+                      // words (fixed offset; zero between calls)
   size_t unit_code;   // int32 [P * d_in]: row << 3 | first_of_group << 2 | plane
   size_t unit_x;      // fp32 [P * d_in]: x_row * 4^(P-1-plane)
   size_t stream_end;  // end of what grinqh_assign writes
@@ -59,13 +65,19 @@ inline WsLayout ws_layout(int d_in, int d_out, int b_max) {
   size_t n_units = (size_t)d_in * P;
   L.tiles = (d_out + kTileOut - 1) / kTileOut;
   L.counters = sizeof(WsHeader);
-  L.unit_code = align256(L.counters + (size_t)kMaxTiles * 4);
+  L.dpartials = align256(L.counters + (size_t)kMaxTiles * 4);
+  L.unit_code = align256(L.dpartials + (size_t)kMaxCtas * kDecodeTileOut * 4);
   L.unit_x = align256(L.unit_code + n_units * 4);
   L.stream_end = align256(L.unit_x + n_units * 4);
   L.partials = L.stream_end;
   L.total = align256(L.partials + (size_t)kMaxCtas * 2 * kTileOut * 4);
   return L;
 }
+
+// End of the workspace's fixed-offset part (header, counters, decode partial words):
+// every call leaves it zero except the error word; after a device error it is
+// cleared again.
+inline size_t ws_fixed_end() { return ws_layout(128, 16, 2).unit_code; }
 
 // ---- precision assignment on 8 consecutive rows (shared by assign and decode) --------
 //
@@ -191,14 +203,13 @@ cudaError_t launch_decode(const uint32_t *planes, const uint16_t *s, const uint1
                           const uint16_t *x, const float *theta, const float *phi, int d_in,
                           int d_out, int b_max, float *y, uint8_t *b, int32_t *lists,
                           int32_t *counts, float *grp_sums, void *ws, cudaStream_t st);
-// The same launch with the split-K state at explicit addresses: `counters` (arrival
-// words, zero; at least ceil(d_out / 1024) of them), `partials` (fp32, kMaxCtas x
-// 1024) and the device error word.
+// The same launch with the split-K state at explicit addresses: `partials`
+// (kMaxCtas x 1024 words, zero; left zero) and the device error word.
 cudaError_t launch_decode_split(const uint32_t *planes, const uint16_t *s, const uint16_t *z,
                                 const uint16_t *x, const float *theta, const float *phi, int d_in,
                                 int d_out, int b_max, float *y, uint8_t *b, int32_t *lists,
-                                int32_t *counts, float *grp_sums, unsigned *counters,
-                                float *partials, int *error, cudaStream_t st);
+                                int32_t *counts, float *grp_sums, float *partials, int *error,
+                                cudaStream_t st);
 // Argument checks of grinqh_decode_gemv (everything but the workspace): GRINQH_OK
 // or the status it returns, with the message set.
 int check_decode_args(const uint32_t *planes, const uint16_t *s, const uint16_t *z,

@@ -8,8 +8,8 @@
 // synchronise the device).  Such a caller cannot provide the workspace that
 // grinqh_decode_gemv needs.  This entry point runs the fused decode kernel
 // (without its optional outputs) and keeps what is neither an input nor the
-// output -- the split-K partial sums, their arrival words and the device
-// error word -- in one fixed-size array that the library reserves
+// output -- the split-K partial sums and the device error word -- in one
+// fixed-size array that the library reserves
 // on every GPU that loads it and holds until the process exits.
 #include <mutex>
 
@@ -18,13 +18,11 @@
 namespace grinqh {
 namespace {
 
-// Scratch layout: the error word (a 256-byte header), the split-K arrival
-// words (one per 1024-output tile: enough for d_out up to 2^24), then the
-// partial sums of up to kMaxCtas CTAs.  None of it depends on d_in, so the
-// scratch serves every shape grinqh_decode_gemv takes.
-constexpr size_t kNaCounters = 256;
-constexpr size_t kNaPartials = kNaCounters + (size_t)((1 << 24) / 1024) * 4;
-constexpr size_t kNoAllocBytes = kNaPartials + (size_t)kMaxCtas * 1024 * 4;  // about 1.2 MB
+// Scratch layout: the error word (a 256-byte header), then the split-K partial
+// words of up to kMaxCtas CTAs (zero between calls).  None of it depends on the
+// shape, so the scratch serves every shape grinqh_decode_gemv takes.
+constexpr size_t kNaPartials = 256;
+constexpr size_t kNoAllocBytes = kNaPartials + (size_t)kMaxCtas * 1024 * 4;  // about 1 MB
 static_assert(kNaPartials % 256 == 0, "aligned regions");
 
 // The scratch.  In host code this name is only a host-side stand-in; kernels
@@ -70,19 +68,12 @@ extern "C" int grinqh_decode_gemv_noalloc(const uint32_t *planes, const uint16_t
     return record_error(GRINQH_ERR_CUDA, "grinqh_decode_gemv_noalloc: scratch address: %s",
                         cudaGetErrorString(e));
   char *sc = static_cast<char *>(base);
-  // Every call shares the array, which keeps the last call's contents.  A
-  // completed call leaves its arrival words at zero, but one that gave up would
-  // not: the words this shape uses are cleared first.  The error word is not:
-  // it keeps the first error until it is read.
-  const size_t tiles = ((size_t)d_out + 1023) / 1024;
-  e = cudaMemsetAsync(sc + kNaCounters, 0, tiles * 4, (cudaStream_t)stream);
-  if (e != cudaSuccess)
-    return record_error(GRINQH_ERR_CUDA, "grinqh_decode_gemv_noalloc: clearing scratch: %s",
-                        cudaGetErrorString(e));
+  // Every call shares the array.  A completed call leaves its partial words at
+  // zero; the error word keeps the first error until it is read (and the read
+  // clears the whole array again).
   e = launch_decode_split(planes, s, z, x, theta, phi, d_in, d_out, b_max, y, nullptr, nullptr,
-                          nullptr, nullptr, reinterpret_cast<unsigned *>(sc + kNaCounters),
-                          reinterpret_cast<float *>(sc + kNaPartials), reinterpret_cast<int *>(sc),
-                          (cudaStream_t)stream);
+                          nullptr, nullptr, reinterpret_cast<float *>(sc + kNaPartials),
+                          reinterpret_cast<int *>(sc), (cudaStream_t)stream);
   if (e != cudaSuccess)
     return record_error(GRINQH_ERR_CUDA, "grinqh_decode_gemv_noalloc launch: %s",
                         cudaGetErrorString(e));
@@ -101,8 +92,8 @@ extern "C" int grinqh_noalloc_check_device_error(void *stream) {
   e = cudaMemcpyAsync(&code, base, sizeof code, cudaMemcpyDeviceToHost, st);
   if (e == cudaSuccess) e = cudaStreamSynchronize(st);
   if (e == cudaSuccess && code != 0) {
-    // clear the error word and the split-K state a failed call may have left
-    e = cudaMemsetAsync(base, 0, kNaPartials, st);
+    // clear the error word and the split-K words a failed call may have left
+    e = cudaMemsetAsync(base, 0, kNoAllocBytes, st);
     if (e == cudaSuccess) e = cudaStreamSynchronize(st);
   }
   if (e != cudaSuccess)

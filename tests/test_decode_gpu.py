@@ -145,39 +145,42 @@ def test_split_k_shares_every_ctas_per_tile(d_out):
     grinqh_check_device_error(lin.ws)  # raises if a split-K wait gave up
 
 
-def test_split_k_wait_gives_up_on_a_stale_arrival_count():
-    # A workspace left with one stale arrival on a tile's arrival word (the call
-    # requires it zeroed): the tile's count completes one arrival early, the CTAs
-    # that arrive after it wait for a count that never comes, give up after their
-    # poll limit, set device error 3 and let the kernel finish; the context stays
-    # usable, and a call on the cleared workspace is right and reports nothing.
+# The fused decode's split-K partial words in a workspace of grinqh_workspace_bytes:
+# after the 256-byte header and grinqh_gemv's arrival counters (one per 512-output
+# tile of the largest d_out, 2^24 / 512 of them), one 1024-word partial per CTA.
+DPARTIALS = 256 + (1 << 24) // 512 * 4
+
+
+def test_split_k_reports_a_partial_word_left_nonzero():
+    # A workspace whose split-K partial words were not left zeroed (the call requires
+    # a zeroed workspace): the first CTA finds its partial's first word non-zero when
+    # it publishes, and the call reports device error 3; the check clears the
+    # workspace's split-K state, and the next call is right and reports nothing.
     from input_adaptive_bit_b200 import ERR_DEVICE, GrinqhError, grinqh_check_device_error
     q, s, z, x, theta = cheap_case(9, 512, 1024, 8)  # one tile: every GEMV CTA shares it
     lin = GrinqhLinear(q, s, z, 8)
     xd, th = to_dev(x), to_dev(theta)
-    counters = lin.ws[256:260].view(torch.int32)  # the tile's arrival word (after the header)
-    counters.fill_(1)
+    lin.ws[DPARTIALS:DPARTIALS + 4].view(torch.int32).fill_(0x3f800001)  # CTA 0's first word
     lin.decode(xd, th, outputs=False)
     torch.cuda.synchronize()
     with pytest.raises(GrinqhError) as err:
         grinqh_check_device_error(lin.ws)
     assert err.value.status == ERR_DEVICE and "code 3" in str(err.value)
-    lin.ws.zero_()
+    assert not lin.ws[:DPARTIALS + 148 * 4096].any()  # the check cleared the split-K state
     _, out = run_layer(None, None, None, x, theta, 8, lin=lin, path="fused")
     b_ref = check_assign(out, x, theta, 8)
     check_y(out, oracle.pack(q, 8), s, z, x, b_ref, 8)
     grinqh_check_device_error(lin.ws)
-    assert not lin.ws[256:256 + 4 * 64].any()  # every arrival word is back at zero
+    assert not lin.ws[DPARTIALS:DPARTIALS + 256 * 4096].any()  # every partial word is back at zero
 
 
-def test_y_is_right_when_some_ctas_cannot_start_until_others_gave_up():
+def test_y_is_right_while_other_work_holds_some_sms():
     # Other work holds a few SMs (single-thread kernels that sleep ~0.8 s on side
-    # streams: the decode kernel's CTAs need a whole SM each, so those SMs stay shut
-    # to it).  CTAs of the same tiles that are running wait for them, give up after
-    # their poll limit (device error 3), mark the tiles' arrival words and exit; the
-    # late CTAs then run, and each tile's last arrival sees the mark and sums the
-    # whole tile.  y must still be the oracle's.
-    from input_adaptive_bit_b200 import ERR_DEVICE, GrinqhError, grinqh_check_device_error
+    # streams; the decode kernel's CTAs need a whole SM each, so those SMs are shut
+    # to it).  The decode launch is cooperative: it starts once all of its CTAs fit,
+    # so the split-K waits between the CTAs of a tile end and y is the oracle's, with
+    # no device error.
+    from input_adaptive_bit_b200 import grinqh_check_device_error
     q, s, z, x, theta = cheap_case(10, 1024, 4096, 8)  # 4 tiles, 36 CTAs each
     lin = GrinqhLinear(q, s, z, 8)
     xd, th = to_dev(x), to_dev(theta)
@@ -194,11 +197,8 @@ def test_y_is_right_when_some_ctas_cannot_start_until_others_gave_up():
     torch.cuda.synchronize()
     b_ref = oracle.assign(x, theta, 8)
     check_y({"y": y.cpu().numpy().astype(np.float64)}, oracle.pack(q, 8), s, z, x, b_ref, 8)
-    try:
-        grinqh_check_device_error(lin.ws)  # 3 if a wait gave up (expected, not required)
-    except GrinqhError as err:
-        assert err.value.status == ERR_DEVICE and "code 3" in str(err.value)
-    assert not lin.ws[256:256 + 4 * 64].any()  # every arrival word is back at zero
+    grinqh_check_device_error(lin.ws)
+    assert not lin.ws[DPARTIALS:DPARTIALS + 256 * 4096].any()  # every partial word is back at zero
 
 
 @pytest.mark.parametrize("shapes", [
@@ -220,7 +220,7 @@ def test_grouped_launch_matches_the_oracle_per_linear(shapes):
         cases.append((q, s, z, x, theta, b_max, lin, xd, th, y))
     nbytes = grinqh_group_workspace_bytes()
     ws = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
-    for _ in range(2):  # twice: the counters must come back to zero
+    for _ in range(2):  # twice: the split-K words must come back to zero
         grinqh_decode_gemv_group([(c[6].planes, c[6].s, c[6].z, c[7], c[8], None, c[6].d_in,
                                    c[6].d_out, c[5], c[9]) for c in cases], ws, nbytes)
         torch.cuda.synchronize()
@@ -228,7 +228,7 @@ def test_grouped_launch_matches_the_oracle_per_linear(shapes):
             out = {"y": y.cpu().numpy().astype(np.float64)}
             check_y(out, oracle.pack(q, b_max), s, z, x, oracle.assign(x, theta, b_max), b_max)
     grinqh_check_device_error(ws)
-    assert not ws[256:256 + 4 * 64].any()  # every arrival counter is back at zero
+    assert not ws[256:].any()  # every split-K partial word is back at zero
 
 
 def test_decode_group_helper_of_the_layer_module():
