@@ -62,7 +62,7 @@ NCU_TRAFFIC = {
     # gemv.cu, grinqh_gemv
     "84585736bc0dc9cf2ac9f0a4738586346a63ac0a4e44acbdc753bb3917df6db4": 17150844,
     # decode.cu, grinqh_decode_gemv (mean over the 60 launches of five steps)
-    "88d880b4be63b01a731d9e57ce3fe4a9be268a329f0936836767fdab03734c7c": 17346492,
+    "c47d66cfdcd82c55fac824c3559139bcb3f01513339e270ed452c49dc315c372": 17345071,
 }
 KERNEL_SOURCE = {"fused": "decode.cu", "two": "gemv.cu"}
 

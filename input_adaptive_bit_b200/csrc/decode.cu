@@ -21,12 +21,11 @@
 //    other kernel and no global round trip sit between x and the GEMV.  Units
 //    are ordered by group, plane, row.
 //  * The m partial tiles of a tile meet in global memory: every CTA of the tile
-//    publishes its partial, waits until all m have arrived, and adds up its own
-//    1/m share of the outputs over the m partials in CTA order (deterministic).
-//    A CTA that waits too long (another CTA of the tile is not running: the GPU
-//    is shared) marks the tile's arrival word and exits; the tile's last
-//    arrival sees the mark and sums the whole tile, so y never depends on the
-//    CTAs being resident together.
+//    publishes its partial as words that are never zero, then adds up its own
+//    1/m share of the outputs over the m partials in CTA order (deterministic),
+//    polling those words until they are non-zero and zeroing them once read.
+//    The launch is cooperative, so all CTAs of a tile are resident together and
+//    the polls end whatever else runs on the GPU.
 //  * A CTA walks its range in windows of 8 groups and rounds of at most 2048
 //    units.  The segments stream through an 8-stage shared-memory ring
 //    (cp.async, 16 B per thread and copy, one barrier per 64-unit stage).
