@@ -165,3 +165,39 @@ def test_device_error_word_is_kept_until_read():
     b_host = oracle.assign(x, theta, 8)
     y_ref, bound = oracle.gemv(oracle.pack(q, 8), s, z, x, b_host, 8, threads=oracle.max_threads())
     assert _within(y.cpu().numpy(), y_ref, bound)
+
+
+@pytest.mark.gpu
+def test_partial_word_left_nonzero_is_reported_and_cleared():
+    # A split-K partial word left non-zero in the fixed array (as a failed call could
+    # leave it) is found when the first CTA publishes over it: the call records
+    # device error 3, the check reports it and clears the array, and the next call
+    # is right and reports nothing.
+    assert torch.cuda.is_available()
+    g = np.random.default_rng(11)
+    d_in, d_out = 1024, 1024
+    q = g.integers(0, 256, size=(d_in, d_out), dtype=np.uint8)
+    s = (g.random((d_in // 128, d_out)) * 0.01 + 1e-4).astype(np.float16)
+    z = (-(g.random((d_in // 128, d_out)) * 0.5)).astype(np.float16)
+    lin = GrinqhLinear(q, s, z, 8)
+    x = synth.activations(g, d_in)
+    theta = synth.quantile_thresholds(np.abs(x.astype(np.float32)), synth.level_fractions(3.0))
+    xd, td = torch.from_numpy(x).cuda(), torch.from_numpy(theta).cuda()
+    y = torch.empty(d_out, dtype=torch.float32, device="cuda")
+    grinqh_noalloc_check_device_error()  # start from a clean array
+    ptr, nbytes = grinqh_noalloc_scratch()
+    words = torch.as_tensor(_DeviceWords(ptr, nbytes // 4), device="cuda")
+    words[64].fill_(0x3f800001)  # the first partial word of CTA 0 (after the 256-byte header)
+    grinqh_decode_gemv_noalloc(lin.planes, lin.s, lin.z, xd, td, None, d_in, d_out, 8, y)
+    torch.cuda.synchronize()
+    with pytest.raises(GrinqhError) as e:
+        grinqh_noalloc_check_device_error()
+    assert e.value.status == ERR_DEVICE and "code 3" in str(e.value)
+    assert not words.any()  # the check cleared the whole array
+    grinqh_decode_gemv_noalloc(lin.planes, lin.s, lin.z, xd, td, None, d_in, d_out, 8, y)
+    torch.cuda.synchronize()
+    grinqh_noalloc_check_device_error()
+    b_host = oracle.assign(x, theta, 8)
+    y_ref, bound = oracle.gemv(oracle.pack(q, 8), s, z, x, b_host, 8, threads=oracle.max_threads())
+    assert _within(y.cpu().numpy(), y_ref, bound)
+    assert not words.any()  # a completed call leaves its partial words at zero
