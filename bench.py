@@ -727,6 +727,37 @@ PREFILL_SETS = 2  # distinct weight sets, alternated step by step
 PREFILL_SWEEP_T = (1, 16, 64, 128, 256, 512, 1024, 2048)
 
 
+def prefill_point(device, T=128, steps=100):
+    """The prefill GEMM of a T-token block through the four Qwen3-8B projections
+    (the prefill workload's step), timed as in its own bench line, beside cuBLAS
+    fp16 on dense weights of the same shapes; for the decode workload's line."""
+    import torch
+    wl = PrefillWorkload(T, device, 0)
+
+    def run(graphs, i):
+        graphs[i % PREFILL_SETS].replay()
+
+    with torch.cuda.stream(wl.stream):
+        for i in range(5):
+            run(wl.graphs, i)
+        ms = device_time_ms(torch, wl.stream, lambda i: run(wl.graphs, i), steps) / steps
+    dgraphs, keep = wl.dense_graphs()
+    with torch.cuda.stream(wl.stream):
+        for i in range(3):
+            run(dgraphs, i)
+        ms_d = device_time_ms(torch, wl.stream, lambda i: run(dgraphs, i), steps) / steps
+    flops = wl.flops
+    del dgraphs, keep, wl
+    torch.cuda.empty_cache()
+    peak, kind = measured_tensor_peak(sustained=True)
+    tf = flops / (ms * 1e-3) / 1e12
+    return {"tokens": T, "shapes": "q 4096x4096, gate/up 4096x12288, down 12288x4096, b_max 8",
+            "ms_per_step": round(ms, 5), "TFLOPs": round(tf, 1),
+            "frac_of_tensor_peak": round(tf / peak, 4), "peak": peak, "peak_kind": kind,
+            "cublas_fp16_dense_ms": round(ms_d, 5), "time_vs_cublas": round(ms / ms_d, 3),
+            "kernel": "prefill_kernel (grinqh_prefill_gemm)"}
+
+
 def measured_tensor_peak(sustained: bool):
     """Dense 16-bit tensor-core peak in TFLOP/s: the measured cuBLAS bf16 figure
     (fp16 has the same nominal dense rate on B200, ratio 1)."""
@@ -1200,7 +1231,7 @@ def main(argv=None):
     planes_mb = sum(lin.planes.numel() * 4 for lin in wl.layers) // 2**20
     cases = None
     dense4 = None
-    sweep_fit = seventy = small_batch = None
+    sweep_fit = seventy = small_batch = prefill = None
     if not args.no_cases and rank == 0:
         cases = cold_case_times(wl)
         dense4 = dense4_times(wl)
@@ -1211,6 +1242,7 @@ def main(argv=None):
             sweep_fit = uniform_sweep_fit(device)
             seventy = seventy_b_pair(device, peak_hbm)
             small_batch = small_batch_sweep(device)
+            prefill = prefill_point(device)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -1271,6 +1303,8 @@ def main(argv=None):
         line["seventy_b_class"] = seventy
     if small_batch is not None:
         line["small_batch"] = small_batch
+    if prefill is not None:
+        line["prefill"] = prefill
     print(json.dumps(line), flush=True)
     return 0
 
