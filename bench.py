@@ -24,6 +24,12 @@ rank 0.  With --gpus N > 1 (under torchrun) every rank runs its own replica of
 the workload (weak scaling, no collective on the data path); the step time is
 the max over ranks.
 
+Beside the headline, the default line carries the per-GEMV cold-L2 table and
+the dense 4-bit comparator (`cases`, `dense4`), the uniform-width sweep and its
+linear fit (`latency_vs_bits`), a 70B-class pair (`seventy_b_class`), the
+small-batch kernel at B = 2/4/8 (`small_batch`) and one prefill point
+(`prefill`, 128 tokens, with cuBLAS on dense weights beside it).
+
 --workload prefill-qwen3-8b times the other phase instead: a step is the
 prefill GEMM (grinqh_prefill_gemm, every row at the full width b_max = 8) of
 a block of T prompt tokens (default 128) through the same four Qwen3-8B
